@@ -1,0 +1,385 @@
+"""Benchmark of the paged KV cache hot path on B200.
+
+One step = kv_append of every new token (norm, RoPE, 16-bit conversion,
+scatter) followed by paged_decode_attention over every sequence, on the
+Llama-3-8B-shaped batch-32 decode workload (Hq=32, Hkv=8, D=128, bf16 pool,
+block size 16, contexts U[512, 4096]). Inputs are synthetic and seeded.
+
+Reports whole-step KV-read throughput (algorithmic K+V bytes of the decode
+pass divided by the step time), the decode kernel against the measured HBM
+roofline, an end-to-end figure through the C ABI with host buffers, the CPU
+oracle timed on this host, and the SM clocks seen during the timed region.
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+        under torchrun for N > 1 (one rank per GPU, independent replicas).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attn KV-read GB/s (% of HBM peak); seq-steps/s at batch 32"
+WORKLOAD = "llama3-8b-b32"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+DECODE_SOURCES = ("paged_kv_cache_321_b200/csrc/decode.cu", "paged_kv_cache_321_b200/csrc/common.cuh")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--split-tokens", type=int, default=0)
+    return ap.parse_args()
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def sources_sha(paths) -> str:
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, or None
+    when the kernel sources changed since that capture."""
+    path = os.path.join(ROOT, "profiles", f"decode_{workload}.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    if d.get("sources_sha") != sources_sha(DECODE_SOURCES):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.1)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus: int):
+    import torch
+
+    if n_gpus <= 1 or "RANK" not in os.environ:
+        return 0, 1, None
+    import datetime
+
+    import torch.distributed as dist
+
+    rank, world = int(os.environ["RANK"]), int(os.environ["WORLD_SIZE"])
+    local = int(os.environ.get("LOCAL_RANK", rank))
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                            device_id=torch.device("cuda", local))
+    return rank, world, dist
+
+
+# ------------------------------------------------------------------ oracle
+def oracle_step(orc, wl, seqs, threads):
+    """The oracle's step restricted to the given sequences: their new tokens'
+    append, then their decode attention."""
+    sp = wl.spec
+    tok = wl.cu_q[seqs]
+    pk = wl.pool_k[sp.layer].copy()
+    pv = wl.pool_v[sp.layer].copy()
+    rope = orc.rope_table(float(np.float32(sp.theta)), sp.D, wl.max_seq_len) if sp.theta else None
+    st, q_out = orc.kv_append(Hq=sp.Hq, Hkv=sp.Hkv, D=sp.D, bs=sp.bs, kv_dtype=sp.kv_dtype, q=wl.q[tok], k=wl.k[tok],
+                              v=wl.v[tok], tok_req=wl.tok_req[tok], positions=wl.positions[tok],
+                              block_tables=wl.block_tables, pool_k=pk, pool_v=pv, max_seq_len=wl.max_seq_len,
+                              q_norm_w=wl.q_norm_w, k_norm_w=wl.k_norm_w, eps=sp.eps, rope=rope)
+    st2, out, _ = orc.paged_attention(Hq=sp.Hq, Hkv=sp.Hkv, D=sp.D, bs=sp.bs, kv_dtype=sp.kv_dtype,
+                                      q=q_out.reshape(-1, sp.Hq, sp.D), q_seq=seqs, q_pos=wl.ctx[seqs] - 1,
+                                      block_tables=wl.block_tables, pool_k=pk, pool_v=pv, threads=threads)
+    return st | st2
+
+
+def cpu_baseline(wl, budget_s=12.0):
+    import oracle as orc
+
+    threads = os.cpu_count() or 1
+    seqs = wl.decode_seqs
+    t0 = time.perf_counter()
+    reps, nbytes = 0, 0
+    while True:
+        oracle_step(orc, wl, seqs, threads)
+        reps += 1
+        nbytes += wl.kv_read_bytes(seqs)
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"{reps} full step(s) of {WORKLOAD}: append of {len(seqs)} tokens + fp64 attention over "
+                      f"{len(seqs)} sequences ({wl.kv_read_bytes(seqs) / 1e6:.1f} MB KV each)",
+            "seconds": round(dt, 2)}
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle, as it stands, on this host."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle as orc
+    from workloads import SPECS, make_workload
+
+    wl = make_workload(SPECS[args.workload])
+    threads = os.cpu_count() or 1
+    seqs_all = wl.decode_seqs
+    # size one step so the whole run stays within about two minutes
+    t0 = time.perf_counter()
+    oracle_step(orc, wl, seqs_all[:1], threads)
+    one = time.perf_counter() - t0
+    total = args.steps + args.warmup
+    n = int(max(1, min(len(seqs_all), 120.0 / max(total * one, 1e-9))))
+    seqs = seqs_all[:n]
+    for _ in range(args.warmup):
+        oracle_step(orc, wl, seqs, threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(orc, wl, seqs, threads)
+    dt = time.perf_counter() - t0
+    gbs = wl.kv_read_bytes(seqs) * args.steps / dt / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "sample_sequences": n, "of_sequences": len(seqs_all)},
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{n} of {len(seqs_all)} sequences per step (append + fp64 attention)"},
+        "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------- ours
+def run_ours(args):
+    import torch
+
+    rank, world, dist = dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import paged_kv_cache_321_b200 as K
+    from workloads import SPECS, make_workload
+
+    spec = SPECS[args.workload]
+    wl = make_workload(spec, seed_offset=spec.seed_offset + 1000 * rank)  # one independent replica per rank
+    sp = wl.spec
+    stream = torch.cuda.current_stream()
+
+    pool = K.Pool(sp.num_layers, sp.Hkv, sp.D, sp.bs, wl.max_seq_len, wl.num_blocks, sp.kv_dtype, device=dev)
+    pool.k.copy_(torch.from_numpy(wl.pool_k.view(np.int16)))
+    pool.v.copy_(torch.from_numpy(wl.pool_v.view(np.int16)))
+    attn = K.attn_config(sp.Hq, sp.Hkv, sp.D, float(np.float32(sp.theta)), sp.eps)
+    rope = torch.empty(wl.max_seq_len * sp.D, dtype=torch.float32, device=dev)
+    K.rope_table_fill(attn, wl.max_seq_len, rope)
+    g = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    q, k, v = g(wl.q), g(wl.k), g(wl.v)
+    qn, kn = g(wl.q_norm_w), g(wl.k_norm_w)
+    tok_req, positions, bt, ctx = g(wl.tok_req), g(wl.positions), g(wl.block_tables), g(wl.ctx)
+    seqs = wl.decode_seqs
+    assert len(seqs) == wl.S, "the benchmark workload is decode-only"
+    B, T, mx = wl.S, wl.T, int(wl.ctx.max())
+    q_out = torch.empty((T, sp.Hq * sp.D), dtype=torch.float32, device=dev)
+    out = torch.empty((B, sp.Hq, sp.D), dtype=torch.float32, device=dev)
+    ws_n = K.decode_workspace_size(pool, attn, B, mx, args.split_tokens)
+    ws = torch.zeros(ws_n // 4 + 64, dtype=torch.float32, device=dev)
+    kv_bytes = wl.kv_read_bytes()
+
+    def append():
+        K.kv_append(pool, sp.layer, attn, q, k, v, tok_req, positions, bt, q_out, qn, kn, rope, wl.max_seq_len,
+                    stream=stream)
+
+    def decode():
+        K.paged_decode_attention(pool, sp.layer, attn, q_out.view(B, sp.Hq, sp.D), bt, ctx, mx, out, ws,
+                                 args.split_tokens, stream=stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    # ---- device-resident timing: K steps, events around every decode launch
+    for _ in range(max(args.warmup, 3)):
+        append()
+        decode()
+    pool.sync_status(stream)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        append()
+        ev[i][0].record(stream)
+        decode()
+        ev[i][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    pool.sync_status(stream)
+    step_ms = t_start.elapsed_time(t_end) / args.steps
+    dec_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    if dist is not None:
+        t = torch.tensor([step_ms, dec_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        step_ms, dec_ms = float(t[0]), float(t[1])
+
+    # ---- end to end through the C ABI with host buffers: H2D of the step's
+    # inputs from pinned memory, the step, D2H of the attention output
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+    h_in = [pin(wl.q), pin(wl.k), pin(wl.v), pin(wl.tok_req), pin(wl.positions), pin(wl.block_tables),
+            pin(wl.ctx)]
+    d_in = [q, k, v, tok_req, positions, bt, ctx]
+    h_out = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in h_in)
+    d2h = h_out.numel() * h_out.element_size()
+    e2e_steps = max(1, min(args.steps, 500))
+
+    def e2e_step():
+        for h, d in zip(h_in, d_in):
+            d.copy_(h, non_blocking=True)
+        append()
+        decode()
+        h_out.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if dist is not None:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+    pool.sync_status(stream)
+
+    peak, peak_kind = measured_peaks()
+    total_bytes = kv_bytes * world
+    value = total_bytes / (step_ms * 1e-3) / 1e9
+    achieved = kv_bytes / (dec_ms * 1e-3) / 1e9
+    traffic = ncu_traffic(args.workload)
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(step_ms, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": sp.kv_dtype,
+        "data": "synthetic",
+        "config": {"workload": args.workload, "batch": B, "Hq": sp.Hq, "Hkv": sp.Hkv, "head_dim": sp.D,
+                   "block_size": sp.bs, "kv_dtype": sp.kv_dtype, "ctx_range": [int(wl.ctx.min()), mx],
+                   "kv_bytes_per_step": kv_bytes, "split_tokens": args.split_tokens or "auto",
+                   "l2": f"inputs larger than L2 ({kv_bytes / 1e6:.0f} MB of K/V per step vs 126 MB L2)",
+                   "parallelism": f"replicas x{world}"},
+        "seq_steps_per_s": round(B * world / (step_ms * 1e-3), 1),
+        "decode_attention_gbs": round(achieved * world, 2),
+        "pct_of_measured_hbm": round(100 * achieved / peak, 2),
+        "pct_of_nominal_8tbs": round(100 * achieved / NOMINAL_HBM_GBS, 2),
+        "decode_us": round(dec_ms * 1e3, 2),
+        "append_us_incl_gap": round((step_ms - dec_ms) * 1e3, 2),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "peak_kind": peak_kind, "kernel": "kvp::dec::decode_kernel"},
+        "clocks": clk,
+        "e2e": {"value": round(total_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
+        "gpu_launches": 2 * args.steps,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    pool.close()
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

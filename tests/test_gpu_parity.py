@@ -87,7 +87,10 @@ def test_append_and_decode_small(orc, dev, name):
     q_ref, pk, pv = _check_append(orc, run)
     st, ref = oracle_decode(orc, wl, q_ref, pk, pv)
     assert st == 0
-    for split in (0, 16 * max(1, wl.spec.bs // 16), 0 if wl.spec.bs > 64 else 64):
+    unit = max(16, wl.spec.bs)
+    mx = int(wl.ctx.max())
+    finest = unit * max(1, -(-mx // (unit * 100)))  # the smallest split giving <= 100 splits
+    for split in (0, finest, 4 * finest):
         out = run.decode(split_tokens=split)
         run.pool.sync_status()
         assert_close(out.cpu().numpy(), ref, f"{name} split={split}")
