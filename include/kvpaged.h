@@ -206,6 +206,34 @@ int paged_decode_attention(kvp_pool *pool, int layer, const kvp_attn_config *att
                            int max_ctx_len, int split_tokens, float *out, void *workspace, size_t ws_bytes,
                            void *stream);
 
+/* Size of the fixed workspace of paged_decode_attention_noalloc: 16 MiB. */
+#define KVP_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+/* paged_decode_attention for callers that cannot allocate device memory.
+ * The pages have no counterpart of this entry point. It serves callers that
+ * cannot call cudaMalloc: a host program that reserved all of the GPU's memory
+ * for its own allocator at start-up, or a latency-critical serving loop that
+ * cannot afford cudaMalloc's device-wide synchronisation. Instead of a
+ * caller-provided workspace it uses a fixed array of
+ * KVP_NOALLOC_SCRATCH_BYTES inside the library's device memory, reserved on
+ * every GPU that loads the library and held until the process exits. It
+ * allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *   - Arguments, results and device errors are those of
+ *     paged_decode_attention without workspace / ws_bytes.
+ *   - A call whose workspace (paged_decode_workspace_size with the same B,
+ *     max_ctx_len and split_tokens) exceeds KVP_NOALLOC_SCRATCH_BYTES is
+ *     refused with KVP_EINVAL and a message naming the sizes.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the one array, which keeps the previous
+ *     call's contents; each call clears the split counters on `stream` before
+ *     its launch. Calls that overlap on the GPU (another stream, another
+ *     thread) race on the array and must be serialised by the caller. */
+int paged_decode_attention_noalloc(kvp_pool *pool, int layer, const kvp_attn_config *attn, int B, const float *q,
+                                   const int32_t *block_tables, int max_blocks_per_seq, const int32_t *ctx_lens,
+                                   int max_ctx_len, int split_tokens, float *out, void *stream);
+
 /* ------------------------------------------------------ prefill attention */
 
 /* Workspace bytes paged_prefill_attention needs (0 on a bad argument). */

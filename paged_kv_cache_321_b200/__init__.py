@@ -25,6 +25,8 @@ from ._native import (  # noqa: F401
     kv_append,
     lib,
     paged_decode_attention,
+    paged_decode_attention_noalloc,
+    NOALLOC_SCRATCH_BYTES,
     paged_prefill_attention,
     prefill_workspace_size,
     rope_table_bytes,

@@ -28,7 +28,7 @@ STATUS_NAMES = {0: "KVP_OK", -1: "KVP_EINVAL", -2: "KVP_ERANGE", -3: "KVP_EOVERF
 EXPORTS = (
     "kv_pool_create", "kv_pool_destroy", "kv_pool_layer_ptrs", "kv_pool_sync_status", "kvp_last_error",
     "kvp_rope_table_bytes", "kvp_rope_table_fill", "kv_append", "paged_decode_workspace_size",
-    "paged_decode_attention", "paged_prefill_workspace_size", "paged_prefill_attention", "kvp_convert_f32",
+    "paged_decode_attention", "paged_decode_attention_noalloc", "paged_prefill_workspace_size", "paged_prefill_attention", "kvp_convert_f32",
     "kvp_convert_bits", "kvp_version",
 )
 
@@ -73,6 +73,7 @@ def lib() -> C.CDLL:
             "kv_append": (i32, [P, i32, AP, i32, P, P, P, P, P, P, i32, P, P, i32, P, i32, P, P]),
             "paged_decode_workspace_size": (sz, [P, AP, i32, i32, i32]),
             "paged_decode_attention": (i32, [P, i32, AP, i32, P, P, i32, P, i32, i32, P, P, sz, P]),
+            "paged_decode_attention_noalloc": (i32, [P, i32, AP, i32, P, P, i32, P, i32, i32, P, P]),
             "paged_prefill_workspace_size": (sz, [P, AP, i32, i32, i32]),
             "paged_prefill_attention": (i32, [P, i32, AP, i32, P, P, P, P, i32, i32, i32, P, P, sz, P]),
             "kvp_convert_f32": (i32, [P, P, i64, i32, P]),
@@ -191,6 +192,19 @@ def paged_decode_attention(pool: Pool, layer: int, attn: AttnConfig, q, block_ta
                                         block_tables.shape[1], _ptr(ctx_lens), max_ctx_len, split_tokens, _ptr(out),
                                         _ptr(workspace), workspace.numel() * workspace.element_size(),
                                         _stream(stream)))
+
+
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024  # KVP_NOALLOC_SCRATCH_BYTES
+
+
+def paged_decode_attention_noalloc(pool: Pool, layer: int, attn: AttnConfig, q, block_tables, ctx_lens,
+                                   max_ctx_len: int, out, split_tokens: int = 0, stream=None):
+    """paged_decode_attention using the library's fixed device workspace, for
+    callers that cannot allocate device memory (see include/kvpaged.h)."""
+    B = ctx_lens.numel()
+    _check(lib().paged_decode_attention_noalloc(pool.handle, layer, C.byref(attn), B, _ptr(q), _ptr(block_tables),
+                                                block_tables.shape[1], _ptr(ctx_lens), max_ctx_len, split_tokens,
+                                                _ptr(out), _stream(stream)))
 
 
 def prefill_workspace_size(pool: Pool, attn: AttnConfig, S: int, total_q: int, max_q_len: int) -> int:
