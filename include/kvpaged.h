@@ -185,15 +185,18 @@ size_t paged_decode_workspace_size(const kvp_pool *pool, const kvp_attn_config *
  * token kv_append just wrote:
  *   out[r][g] = sum_j softmax_j(q[r][g] . K_j * scale) V_j,
  *   scale = float32(1/sqrt(float64(D))),
- * accumulated in fp32 with an online softmax; the context is cut into splits
- * of split_tokens keys (0 = automatic; otherwise a multiple of
- * max(16, block_size)), each split's (max, sum, unnormalised output) is
- * combined by log-sum-exp in fp32 by the last split to finish.
+ * accumulated in fp32 with an online softmax over 16-key tiles. The tiles of
+ * all (sequence, kv head) contexts are divided evenly among the GPU's warps;
+ * a context shared by several warps is combined from their (max, sum,
+ * unnormalised output) partials by log-sum-exp in fp32 by the last of them to
+ * finish. split_tokens is the fewest keys one warp takes (0 = automatic;
+ * otherwise a multiple of 16): a large value keeps each context on one warp.
  *
  *   q, out        [B][Hq][D] float32
  *   block_tables  [B][max_blocks_per_seq] int32 (entries past the context are
  *                 never read)
  *   ctx_lens      [B] int32 in [0, max_ctx_len]; 0 gives an all-zero row
+ *   B             at most 2048
  *   workspace     >= paged_decode_workspace_size(...) bytes, 256-byte
  *                 aligned, ZERO-FILLED before its first use; every call leaves
  *                 its counters at zero again. Calls sharing a workspace must

@@ -1,5 +1,5 @@
 // paged_decode_attention: one query token per sequence, GQA attention over a
-// block-pooled KV cache, with split-K over the context.
+// block-pooled KV cache, split over the context with a log-sum-exp combine.
 //
 // Method: the batch kernel of runHybridAttentionBlockBatch in
 // makarna/pkg/model/arch/hybrid_decoder.go (one query per request, per-request
@@ -8,29 +8,31 @@
 // soft3/glia/run/arch/decoder/forward.rs (kv head = h / (Hq/Hkv), max-subtracted
 // softmax, sum of p * v), computed as an online softmax over 16-token tiles.
 //
-// B200 design (HBM-bound: every K/V byte is read once, ~4-8 flop per byte):
-//  * grid (split, kv head, sequence); one CTA streams one split of one
-//    (sequence, kv head) and serves all G query heads of that kv head from a
-//    single read of K and V;
-//  * 4 warps per CTA, each with a private 2-stage ring of 16-token tiles. A
-//    tile of K (and of V) for one head is one contiguous run of the
-//    head-major pool, fetched by ONE 1-D bulk async copy (cp.async.bulk, TMA
-//    engine, no multicast) that completes on the stage's mbarrier, so no
-//    registers are spent on loads in flight;
-//  * each token is handled by LPT lanes; lane j of a token owns DPL dims
-//    (16-byte shared-memory chunks j, j+LPT, ..., conflict-free) and keeps
-//    q (pre-scaled by scale*log2(e)) and the output accumulators for all G
-//    heads in registers; products use packed f32x2 FMAs;
-//  * the G partial dot products of a token are summed across its LPT lanes
-//    by a transposed butterfly (each step halves the values per lane), which
-//    leaves lane j holding the full score of head j >> HSHIFT;
-//  * per tile: one max, one rescale of the accumulators (skipped when no
-//    head's max moved), exp2 of the scores, P broadcast through shared
-//    memory, P.V;
-//  * the CTA's 4 warps are merged in shared memory; a CTA whose split is not
-//    the only one writes (max, sum, unnormalised output) to the workspace and
-//    bumps the (sequence, head) counter; the last split to finish combines
-//    all partials by log-sum-exp and resets the counter (no second launch).
+// B200 design. The step is HBM-bound (every K/V byte is read once, ~4-8 flop
+// per byte on CUDA cores), so the kernel is built to keep bytes in flight and
+// the issue slots busy:
+//  * persistent: one CTA per SM, NW independent warps. The tiles of all
+//    (sequence, kv head) contexts, taken in order, form one global sequence
+//    that is cut into equal contiguous ranges, one per warp (stream-K), so the
+//    load is balanced to one tile whatever the context lengths;
+//  * each warp streams its range through a private ring of NST stages; a
+//    stage holds one 16-token tile of K and of V for one head, each fetched by
+//    ONE 1-D bulk async copy (cp.async.bulk on the TMA engine, no multicast)
+//    completing on the stage's mbarrier. The ring runs on across context
+//    boundaries, so the next context's tiles are in flight while the current
+//    one is finished;
+//  * LPT lanes per token, each owning DPL dims (16-byte chunks j, j+LPT, ...:
+//    conflict-free shared-memory reads); q (pre-scaled by scale*log2 e) and
+//    the output accumulators for all G heads of the kv head stay in
+//    registers; products are packed f32x2 FMAs;
+//  * the partial dot products of a pass (ITERS tokens x G heads) are summed
+//    over the LPT lanes by one batched transposed butterfly that halves the
+//    values at every step, leaving each lane with distinct (token, head)
+//    scores; one exp2 per score, P goes to the PV pass through shared memory;
+//  * a context split over several warps leaves (max, sum, unnormalised
+//    output) partials in the workspace; the warp that finishes the context
+//    last (atomic counter) combines them by log-sum-exp and resets the
+//    counter, so no second launch is needed.
 #include <math.h>
 
 #include "common.cuh"
@@ -38,27 +40,40 @@
 namespace kvp {
 namespace dec {
 
-constexpr int NW = 4;   // warps per CTA
-constexpr int TT = 16;  // tokens per tile (stage)
-constexpr int NST = 2;  // stages per warp
-constexpr int kMaxSplits = 128;
+constexpr int TT = 16;             // tokens per tile (stage)
+constexpr int NST = 2;             // stages per warp
+constexpr int kMaxBatch = 2048;    // sequences per call (per-CTA prefix in shared memory)
+constexpr int kAutoMinTiles = 2;   // default minimum tiles per warp
+constexpr int kStageBudget = 200 * 1024;
 
 constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
+constexpr int cmin(int a, int b) { return a < b ? a : b; }
+constexpr int cmax(int a, int b) { return a > b ? a : b; }
 
 template <int D, int G>
 struct Shape {
-    static constexpr int DPL = (G <= 4 && D >= 128) ? 16 : 8;  // dims per lane
+    static constexpr int DPL = 8;                                // dims per lane (one 16-byte chunk)
     static constexpr int LPT = D / DPL;                          // lanes per token
     static constexpr int TPW = 32 / LPT;                         // tokens per warp pass
-    static constexpr int CH = DPL / 8;                           // 16-byte chunks per lane per row
     static constexpr int ITERS = TT / TPW;                       // passes per tile
-    static constexpr int HSHIFT = ilog2(LPT) - ilog2(G);         // lane j -> head j >> HSHIFT
+    static constexpr int RB = cmin(ITERS, cmax(1, 32 / G));      // passes reduced together
+    static constexpr int NB = ITERS / RB;                        // reduction batches per tile
+    static constexpr int NV = RB * G;                            // partial sums per lane per batch
+    static constexpr int LEVELS = ilog2(LPT);                    // butterfly steps over a token's lanes
+    static constexpr int HALV = cmin(LEVELS, ilog2(RB));         // steps that halve the passes kept
+    static constexpr int PPL = RB >> HALV;                       // passes a lane keeps per batch
+    static constexpr int REP = 1 << (LEVELS - HALV);             // lanes holding copies of a score
     static constexpr int TILE_WORDS = TT * D;                    // 16-bit words of K (or V) per tile
-    static constexpr int STAGE_WORDS = 2 * TILE_WORDS;
-    static constexpr int STAGE_BYTES_ALL = NW * NST * STAGE_WORDS * 2;
+    static constexpr int STAGE_BYTES = 2 * TILE_WORDS * 2;
+    static constexpr int NO = G * DPL / 2;                       // float2 output accumulators per lane
+    static constexpr int OLEV = ilog2(TPW);
+    static constexpr int OVPL = NO >> OLEV;                      // float2 outputs a lane owns
+    // warps per CTA (one CTA per SM): within the register budget and the
+    // shared-memory budget of the stage rings
+    static constexpr int NW = cmin(G >= 8 ? 8 : 12, kStageBudget / (NST * STAGE_BYTES));
     static_assert(LPT >= 8 && LPT <= 32, "lanes per token");
-    static_assert(HSHIFT >= 0, "group larger than lanes per token");
-    static_assert(NW * TPW * G * D * 4 <= STAGE_BYTES_ALL, "combine area");
+    static_assert(ITERS % RB == 0, "reduction batches");
+    static_assert(ilog2(NO) >= OLEV, "token-group reduction must halve at every step");
 };
 
 struct Params {
@@ -67,11 +82,10 @@ struct Params {
     const int32_t *bt;        // [B][mbps]
     const int32_t *ctx;       // [B]
     float *out;               // [B][Hq][D]
-    float *ws_ml;             // [B][Hkv][max_splits][G][2]
-    float *ws_o;              // [B][Hkv][max_splits][G][D]
-    int *counters;            // [B][Hkv]
+    float *part;              // [W + B*Hkv][G][D + 2]: output, then (max, sum) per head
+    int *counters;            // [B*Hkv]
     int *status;
-    int Hq, Hkv, mbps, bs, num_blocks, max_ctx, max_seq_len, split, max_splits, chunk_blocks;
+    int B, Hq, Hkv, mbps, bs, num_blocks, max_ctx, max_seq_len, warps_total, min_tiles;
     float qscale;  // softmax scale * log2(e)
 };
 
@@ -81,14 +95,26 @@ template <int D, int G>
 struct Smem {
     using S = Shape<D, G>;
     static constexpr size_t stages = 0;
-    static constexpr size_t bars = S::STAGE_BYTES_ALL;
-    static constexpr size_t masks = bars + NW * NST * 8;
-    static constexpr size_t pbuf = align_up(masks + NW * NST * 4, 16);
-    static constexpr size_t cm = pbuf + NW * TT * G * 4;  // per-warp (max, sum), aliased later
-    static constexpr size_t flag = align_up(cm + 2 * NW * G * 4, 16);
-    static constexpr size_t bids = flag + 16;
-    static size_t total(int chunk_blocks) { return align_up(bids + 4 * static_cast<size_t>(chunk_blocks), 128); }
+    static constexpr size_t bars = static_cast<size_t>(S::NW) * NST * S::STAGE_BYTES;
+    static constexpr size_t masks = bars + S::NW * NST * 8;
+    static constexpr size_t pbuf = align_up(masks + S::NW * NST * 4, 16);
+    static constexpr size_t tiles = pbuf + S::NW * TT * G * 8;  // [B] tiles per sequence
+    __host__ __device__ static size_t pref(int B) { return align_up(tiles + 4 * static_cast<size_t>(B), 16); }  // [B + 1]
+    __host__ __device__ static size_t total(int B) { return align_up(pref(B) + 4 * static_cast<size_t>(B + 1), 128); }
 };
+
+__device__ __forceinline__ float ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float shfl_xor(float x, int off) { return __shfl_xor_sync(0xffffffffu, x, off); }
+__device__ __forceinline__ float2 shfl_xor(float2 x, int off)
+{
+    return make_float2(__shfl_xor_sync(0xffffffffu, x.x, off), __shfl_xor_sync(0xffffffffu, x.y, off));
+}
 
 template <bool BF16>
 __device__ __forceinline__ void unpack8(const uint4 w, float2 (&f)[4])
@@ -99,148 +125,244 @@ __device__ __forceinline__ void unpack8(const uint4 w, float2 (&f)[4])
     f[3] = unpack2<BF16>(w.w);
 }
 
-// Sums v[0..G) over the LPT lanes of a token group; afterwards v[0] of lane j
-// holds the total of head j >> HSHIFT.
-template <int G, int LPT>
-__device__ __forceinline__ void transposed_reduce(float (&v)[G], int j)
+// First value index a lane keeps after HALV halving steps over the lane bits
+// lo_off, 2*lo_off, ... starting from N values.
+template <int N, int HALV>
+__device__ __forceinline__ int halving_base(int lane, int lo_off)
 {
-    int n = G;
+    int base = 0, n = N, off = lo_off;
 #pragma unroll
-    for (int off = LPT / 2; off >= 1; off >>= 1) {
-        if (n > 1) {
-            const bool up = (j & off) != 0;
+    for (int s = 0; s < HALV; ++s) {
+        n >>= 1;
+        if (lane & off) base += n;
+        off <<= 1;
+    }
+    return base;
+}
+
+// Reduces v[0..N) with `op` over the lanes that differ in bits lo_off,
+// 2*lo_off, ... below lim_off. The first HALV steps halve the values a lane
+// keeps (the half chosen by its lane bit, the other half is sent to the
+// partner); later steps combine the single remaining value. Afterwards
+// v[0 .. N >> HALV) hold the complete results for value indices
+// halving_base<N, HALV>(lane, lo_off) + 0, 1, ...
+template <int N, int HALV, typename T, typename Op>
+__device__ __forceinline__ void transposed_reduce(T (&v)[N], int lane, int lo_off, int lim_off, Op op)
+{
+    int n = N;
+    int off = lo_off;
+#pragma unroll
+    for (int step = 0; step < 5; ++step) {
+        if (off >= lim_off) break;
+        if (step < HALV) {
+            const bool up = (lane & off) != 0;
             const int half = n / 2;
 #pragma unroll
-            for (int k = 0; k < G / 2; ++k) {
+            for (int k = 0; k < N / 2; ++k) {
                 if (k < half) {
-                    const float send = up ? v[k] : v[k + half];
-                    const float keep = up ? v[k + half] : v[k];
-                    v[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+                    const T send = up ? v[k] : v[k + half];
+                    const T keep = up ? v[k + half] : v[k];
+                    v[k] = op(keep, shfl_xor(send, off));
                 }
             }
             n = half;
         } else {
-            v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
+            v[0] = op(v[0], shfl_xor(v[0], off));
         }
+        off <<= 1;
+    }
+}
+
+// Position of a warp's cursor in the global tile sequence.
+struct Cursor {
+    int t;   // global tile index
+    int r;   // sequence
+    int h;   // kv head
+    int ti;  // tile index inside the (r, h) context
+    int nt;  // tiles of sequence r
+};
+
+// Log-sum-exp combine of the partials of context (r, h), written by warps
+// w_first .. w_last into consecutive slots; one warp.
+template <int D, int G>
+__device__ void combine(const Params &p, int rhidx, int w_first, int w_last, int lane, float *out_rh)
+{
+    constexpr int SL = G * (D + 2);
+    constexpr int DL = D / 32;  // dims per lane: 2, 4 or 8
+    const int nseg = w_last - w_first + 1;
+    const float *base = p.part + static_cast<size_t>(w_first + rhidx) * SL;
+#pragma unroll 1
+    for (int g = 0; g < G; ++g) {
+        float M = -INFINITY;
+        for (int s = lane; s < nseg; s += 32) M = fmaxf(M, __ldcg(base + static_cast<size_t>(s) * SL + G * D + 2 * g));
+#pragma unroll
+        for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+        float L = 0.0f;
+        for (int s = lane; s < nseg; s += 32) {
+            const float *ml = base + static_cast<size_t>(s) * SL + G * D + 2 * g;
+            const float m = __ldcg(ml);
+            L += (m == -INFINITY) ? 0.0f : __ldcg(ml + 1) * ex2(m - M);
+        }
+#pragma unroll
+        for (int off = 16; off; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+        const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+        float acc[DL];
+#pragma unroll
+        for (int d = 0; d < DL; ++d) acc[d] = 0.0f;
+#pragma unroll 4
+        for (int s = 0; s < nseg; ++s) {
+            const float *sl = base + static_cast<size_t>(s) * SL;
+            const float m = __ldcg(sl + G * D + 2 * g);
+            const float wgt = (m == -INFINITY) ? 0.0f : ex2(m - M);
+            const float *src = sl + g * D + lane * DL;
+#pragma unroll
+            for (int d = 0; d < DL; d += 2) {
+                const float2 v = __ldcg(reinterpret_cast<const float2 *>(src + d));
+                acc[d] += v.x * wgt;
+                acc[d + 1] += v.y * wgt;
+            }
+        }
+#pragma unroll
+        for (int d = 0; d < DL; d += 2)
+            *reinterpret_cast<float2 *>(out_rh + g * D + lane * DL + d) = make_float2(acc[d] * inv, acc[d + 1] * inv);
     }
 }
 
 template <int D, int G, bool BF16>
-__global__ void __launch_bounds__(NW * 32, 3) decode_kernel(const Params p)
+__global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const Params p)
 {
     using S = Shape<D, G>;
     using M = Smem<D, G>;
-    constexpr int DPL = S::DPL, LPT = S::LPT, TPW = S::TPW, CH = S::CH, ITERS = S::ITERS;
+    constexpr int NW = S::NW;
+    constexpr int LPT = S::LPT, TPW = S::TPW, ITERS = S::ITERS;
+    constexpr int RB = S::RB, NB = S::NB, NV = S::NV, HALV = S::HALV, PPL = S::PPL;
     extern __shared__ __align__(128) unsigned char smem[];
     uint16_t *stages = reinterpret_cast<uint16_t *>(smem + M::stages);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + M::bars);
     uint32_t *masks = reinterpret_cast<uint32_t *>(smem + M::masks);
-    float *pbuf = reinterpret_cast<float *>(smem + M::pbuf);
-    float *cm_m = reinterpret_cast<float *>(smem + M::cm);
-    float *cm_l = cm_m + NW * G;
-    int *sflag = reinterpret_cast<int *>(smem + M::flag);
-    int *bids = reinterpret_cast<int *>(smem + M::bids);
+    float2 *pbuf = reinterpret_cast<float2 *>(smem + M::pbuf);
+    int *s_tiles = reinterpret_cast<int *>(smem + M::tiles);
+    int *s_pref = reinterpret_cast<int *>(smem + M::pref(p.B));
 
-    const int split = blockIdx.x, h = blockIdx.y, r = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int ctx = p.ctx[r];
-    float *out_rh = p.out + (static_cast<size_t>(r) * p.Hq + static_cast<size_t>(h) * G) * D;
+    const int B = p.B, Hkv = p.Hkv;
 
-    const bool bad = ctx < 0 || ctx > p.max_ctx || ctx > p.mbps * p.bs || ctx > p.max_seq_len;
-    if (bad || ctx == 0) {
-        if (split == 0) {
-            if (bad && tid == 0) report(p.status, KVP_ERANGE, r);
-            for (int i = tid; i < G * D; i += NW * 32) out_rh[i] = 0.0f;
+    // ---- tiles per sequence; invalid or empty sequences get none and a zero row
+    for (int i = tid; i < B; i += NW * 32) {
+        const int c = p.ctx[i];
+        const bool ok = c >= 0 && c <= p.max_ctx && c <= p.mbps * p.bs && c <= p.max_seq_len;
+        s_tiles[i] = ok ? (c + TT - 1) / TT : 0;
+        if (blockIdx.x == 0 && (!ok || c == 0)) {
+            if (!ok) report(p.status, KVP_ERANGE, i);
+            float4 *o = reinterpret_cast<float4 *>(p.out + static_cast<size_t>(i) * p.Hq * D);
+            for (int k = 0; k < p.Hq * D / 4; ++k) o[k] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        return;
     }
-    const int nsplit = (ctx + p.split - 1) / p.split;
-    if (split >= nsplit) return;
-    const int tok0 = split * p.split;
-    const int tok1 = min(ctx, tok0 + p.split);
-    const int ntiles = (tok1 - tok0 + TT - 1) / TT;
-    const int blk0 = tok0 / p.bs;
-    const int nblk = (tok1 - 1) / p.bs - blk0 + 1;
-    const int32_t *bt_row = p.bt + static_cast<size_t>(r) * p.mbps;
-    for (int i = tid; i < nblk; i += NW * 32) bids[i] = bt_row[blk0 + i];
-    if (tid < NW * NST) mbar_init(smem_addr(&bars[tid]), 1);
-    mbar_init_fence();
+    __syncthreads();
+    // ---- exclusive prefix of tiles * Hkv over the sequences (warp 0)
+    if (warp == 0) {
+        int run = 0;
+        for (int base = 0; base < B; base += 32) {
+            const int i = base + lane;
+            const int v = i < B ? s_tiles[i] * Hkv : 0;
+            int x = v;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, x, off);
+                if (lane >= off) x += y;
+            }
+            if (i < B) s_pref[i] = run + x - v;
+            run += __shfl_sync(0xffffffffu, x, 31);
+        }
+        if (lane == 0) s_pref[B] = run;
+    }
     __syncthreads();
 
-    // ---- per-lane state
-    const int grp = lane / LPT, j = lane % LPT;
-    const int hl = j >> S::HSHIFT;  // head whose score this lane ends up holding
-    float2 q2[G][DPL / 2];
-    {
-        const float *qb = p.q + (static_cast<size_t>(r) * p.Hq + static_cast<size_t>(h) * G) * D;
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-            for (int c = 0; c < CH; ++c) {
-                const float4 *src = reinterpret_cast<const float4 *>(qb + g * D + (j + c * LPT) * 8);
-                const float4 a = src[0], b = src[1];
-                q2[g][c * 4 + 0] = make_float2(a.x * p.qscale, a.y * p.qscale);
-                q2[g][c * 4 + 1] = make_float2(a.z * p.qscale, a.w * p.qscale);
-                q2[g][c * 4 + 2] = make_float2(b.x * p.qscale, b.y * p.qscale);
-                q2[g][c * 4 + 3] = make_float2(b.z * p.qscale, b.w * p.qscale);
-            }
-    }
-    float2 o2[G][DPL / 2];
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-        for (int k = 0; k < DPL / 2; ++k) o2[g][k] = make_float2(0.0f, 0.0f);
-    float m_run[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) m_run[g] = -INFINITY;
-    float l_run = 0.0f;
+    // ---- this warp's share of the global tile sequence
+    const int total = s_pref[B];
+    const int W = max(1, min(p.warps_total, (total + p.min_tiles - 1) / p.min_tiles));
+    const int w = blockIdx.x * NW + warp;
+    if (w >= W) return;
+    const int t_begin = static_cast<int>(static_cast<int64_t>(w) * total / W);
+    const int t_end = static_cast<int>(static_cast<int64_t>(w + 1) * total / W);
+    if (t_begin >= t_end) return;  // no CTA-wide barrier follows
 
-    // ---- this warp's tiles: warp, warp + NW, ...
-    const int nt_w = ntiles > warp ? (ntiles - warp + NW - 1) / NW : 0;
-    uint16_t *wst = stages + static_cast<size_t>(warp) * NST * S::STAGE_WORDS;
     const uint32_t bar0 = smem_addr(&bars[warp * NST]);
-    const size_t head_off = static_cast<size_t>(h) * p.bs * D;
-    const size_t blk_stride = static_cast<size_t>(p.Hkv) * p.bs * D;
+    if (lane < NST) mbar_init(bar0 + lane * 8, 1);
+    mbar_init_fence();
+    __syncwarp();
 
-    // Issues the copies of this warp's i-th tile into stage i % NST (lane 0).
-    auto issue = [&](int i) {
-        const int st = i % NST;
-        const int tb = tok0 + (warp + i * NW) * TT;
+    auto locate = [&](int t, Cursor &c) {
+        int lo = 0, hi = B;  // s_pref[lo] <= t < s_pref[hi]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (s_pref[mid] <= t) lo = mid;
+            else hi = mid;
+        }
+        c.t = t;
+        c.r = lo;
+        c.nt = s_tiles[lo];
+        const int local = t - s_pref[lo];
+        c.h = local / c.nt;
+        c.ti = local - c.h * c.nt;
+    };
+    auto advance = [&](Cursor &c) {
+        ++c.t;
+        if (++c.ti == c.nt) {
+            c.ti = 0;
+            if (++c.h == Hkv) {
+                c.h = 0;
+                do {
+                    ++c.r;
+                } while (c.r < B && s_tiles[c.r] == 0);
+                if (c.r < B) c.nt = s_tiles[c.r];
+            }
+        }
+    };
+
+    uint16_t *wst = stages + static_cast<size_t>(warp) * NST * (S::STAGE_BYTES / 2);
+    float2 *pw = pbuf + warp * TT * G;  // (p, p) pairs per (token, head)
+    const size_t blk_stride = static_cast<size_t>(Hkv) * p.bs * D;
+    const bool big_blocks = p.bs >= TT;  // one block per tile
+
+    // Copies tile c into stage st (lane 0 only). For big blocks the tile's
+    // block id and context length come prefetched (blk, ctx).
+    auto issue = [&](const Cursor &c, int st, int blk, int ctx) {
+        const int tb = c.ti * TT;
         const uint32_t bar = bar0 + st * 8;
-        uint16_t *dk = wst + st * S::STAGE_WORDS;
+        uint16_t *dk = wst + st * (S::STAGE_BYTES / 2);
         uint16_t *dv = dk + S::TILE_WORDS;
+        const size_t head_off = static_cast<size_t>(c.h) * p.bs * D;
         uint32_t mask = 0;
-        if (p.bs >= TT) {
-            const int blk = bids[tb / p.bs - blk0];
-            const int nvalid = min(TT, tok1 - tb);
+        if (big_blocks) {
             if (blk >= 0 && blk < p.num_blocks) {
-                mask = (1u << nvalid) - 1u;
+                mask = (1u << min(TT, ctx - tb)) - 1u;
                 const size_t off = blk * blk_stride + head_off + static_cast<size_t>(tb % p.bs) * D;
-                mbar_arrive_expect_tx(bar, 2 * S::TILE_WORDS * 2);
+                mbar_arrive_expect_tx(bar, S::STAGE_BYTES);
                 bulk_g2s(smem_addr(dk), p.kp + off, S::TILE_WORDS * 2, bar);
                 bulk_g2s(smem_addr(dv), p.vp + off, S::TILE_WORDS * 2, bar);
             } else {
-                report(p.status, KVP_ERANGE, r);
+                report(p.status, KVP_ERANGE, c.r);
                 mbar_arrive(bar);
             }
         } else {
+            const int32_t *btr = p.bt + static_cast<size_t>(c.r) * p.mbps;
             uint32_t bytes = 0;
-            for (int t = 0; t < TT && tb + t < tok1; t += p.bs) {
-                const int blk = bids[(tb + t) / p.bs - blk0];
-                if (blk >= 0 && blk < p.num_blocks) {
+            for (int t = 0; t < TT && tb + t < ctx; t += p.bs) {
+                const int b = btr[(tb + t) / p.bs];
+                if (b >= 0 && b < p.num_blocks) {
                     bytes += 2 * p.bs * D * 2;
-                    const int nv = min(p.bs, tok1 - tb - t);
-                    mask |= ((1u << nv) - 1u) << t;
+                    mask |= ((1u << min(p.bs, ctx - tb - t)) - 1u) << t;
                 } else {
-                    report(p.status, KVP_ERANGE, r);
+                    report(p.status, KVP_ERANGE, c.r);
                 }
             }
             if (bytes) {
                 mbar_arrive_expect_tx(bar, bytes);
-                for (int t = 0; t < TT && tb + t < tok1; t += p.bs) {
-                    const int blk = bids[(tb + t) / p.bs - blk0];
-                    if (blk >= 0 && blk < p.num_blocks) {
-                        const size_t off = blk * blk_stride + head_off;
+                for (int t = 0; t < TT && tb + t < ctx; t += p.bs) {
+                    const int b = btr[(tb + t) / p.bs];
+                    if (b >= 0 && b < p.num_blocks) {
+                        const size_t off = b * blk_stride + head_off;
                         bulk_g2s(smem_addr(dk + t * D), p.kp + off, p.bs * D * 2, bar);
                         bulk_g2s(smem_addr(dv + t * D), p.vp + off, p.bs * D * 2, bar);
                     }
@@ -251,85 +373,178 @@ __global__ void __launch_bounds__(NW * 32, 3) decode_kernel(const Params p)
         }
         masks[warp * NST + st] = mask;
     };
+    // block id and context length of tile c (lane 0; plain loads, used one issue later)
+    auto fetch = [&](const Cursor &c, int &blk, int &ctx) {
+        ctx = p.ctx[c.r];
+        blk = big_blocks ? p.bt[static_cast<size_t>(c.r) * p.mbps + (c.ti * TT) / p.bs] : 0;
+    };
 
-    if (lane == 0)
-        for (int i = 0; i < NST && i < nt_w; ++i) issue(i);
+    Cursor prod, cons;
+    locate(t_begin, prod);
+    cons = prod;
+    int pseq = 0;
+    int pf_blk = 0, pf_ctx = 0;  // prefetched for the next tile to issue (lane 0)
+    for (int i = 0; i < NST && prod.t < t_end; ++i) {
+        if (lane == 0) {
+            int blk, ctx;
+            fetch(prod, blk, ctx);
+            issue(prod, i, blk, ctx);
+        }
+        advance(prod);
+        ++pseq;
+    }
+    if (lane == 0 && prod.t < t_end) fetch(prod, pf_blk, pf_ctx);
     __syncwarp();
 
-    float *pw = pbuf + warp * TT * G;
-    for (int i = 0; i < nt_w; ++i) {
-        const int st = i % NST;
-        const bool done = mbar_wait_bounded(bar0 + st * 8, (i / NST) & 1);
-        if (!__all_sync(0xffffffffu, done)) {
-            if (lane == 0) report(p.status, KVP_ETIMEOUT, r);
-            break;
-        }
-        const uint32_t mask = masks[warp * NST + st];
-        const uint16_t *sk = wst + st * S::STAGE_WORDS;
-        const uint16_t *sv = sk + S::TILE_WORDS;
-        if (mask) {
-            // ---- scores: lane holds head hl's score for tokens it*TPW + grp
-            float sc[ITERS];
+    // ---- per-lane state
+    const int grp = lane / LPT, j = lane % LPT;
+    // The passes of a batch are split over the token's lanes: lane j keeps
+    // passes ppass .. ppass + PPL - 1 after the butterfly, and computes the
+    // pass in slot sp as pass sp ^ ppass so that every butterfly step sends
+    // the upper half of its slots (no per-lane selects).
+    int ppass = 0;
 #pragma unroll
-            for (int it = 0; it < ITERS; ++it) {
-                const int tok = it * TPW + grp;
-                const uint16_t *krow = sk + tok * D;
-                float2 acc[G];
-#pragma unroll
-                for (int g = 0; g < G; ++g) acc[g] = make_float2(0.0f, 0.0f);
-#pragma unroll
-                for (int c = 0; c < CH; ++c) {
-                    const uint4 w = *reinterpret_cast<const uint4 *>(krow + (j + c * LPT) * 8);
-                    float2 kf[4];
-                    unpack8<BF16>(w, kf);
-#pragma unroll
-                    for (int g = 0; g < G; ++g)
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) acc[g] = __ffma2_rn(q2[g][c * 4 + e], kf[e], acc[g]);
-                }
-                float v[G];
-#pragma unroll
-                for (int g = 0; g < G; ++g) v[g] = acc[g].x + acc[g].y;
-                transposed_reduce<G, LPT>(v, j);
-                sc[it] = ((mask >> tok) & 1u) ? v[0] : -INFINITY;
-            }
-            // ---- tile max per head, new running max, rescale factors
-            float mt = sc[0];
-#pragma unroll
-            for (int it = 1; it < ITERS; ++it) mt = fmaxf(mt, sc[it]);
-#pragma unroll
-            for (int off = LPT; off < 32; off <<= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
-            float alpha[G];
-            bool moved = false;
-            float m_me = 0.0f, a_me = 1.0f;
+    for (int l = 0; l < HALV; ++l)
+        if (j & (1 << l)) ppass |= RB >> (l + 1);
+    const bool primary = ((j >> HALV) & (S::REP - 1)) == 0;  // one of the REP copies
+    float2 q2[G][4];
+    float2 o2[G][4];
+    float m_run[G], l_run[G];
+
+    for (int seq = 0; cons.t < t_end; ++seq) {
+        if (cons.t == t_begin || cons.ti == 0) {  // a new context segment starts
+            const float *qb = p.q + (static_cast<size_t>(cons.r) * p.Hq + static_cast<size_t>(cons.h) * G) * D + j * 8;
 #pragma unroll
             for (int g = 0; g < G; ++g) {
-                const float mg = __shfl_sync(0xffffffffu, mt, g << S::HSHIFT);
-                const float mn = fmaxf(m_run[g], mg);
-                alpha[g] = (mn == m_run[g]) ? 1.0f : exp2f(m_run[g] - mn);
+                const float4 *src = reinterpret_cast<const float4 *>(qb + g * D);
+                const float4 a = __ldg(src), b = __ldg(src + 1);
+                q2[g][0] = make_float2(a.x * p.qscale, a.y * p.qscale);
+                q2[g][1] = make_float2(a.z * p.qscale, a.w * p.qscale);
+                q2[g][2] = make_float2(b.x * p.qscale, b.y * p.qscale);
+                q2[g][3] = make_float2(b.z * p.qscale, b.w * p.qscale);
+                m_run[g] = -INFINITY;
+                l_run[g] = 0.0f;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) o2[g][k] = make_float2(0.0f, 0.0f);
+            }
+        }
+
+        const int st = seq % NST;
+        const bool done = mbar_wait_bounded(bar0 + st * 8, (seq / NST) & 1);
+        if (!__all_sync(0xffffffffu, done)) {
+            if (lane == 0) report(p.status, KVP_ETIMEOUT, cons.r);
+            return;
+        }
+        const uint32_t mask = masks[warp * NST + st];
+        const uint16_t *sk = wst + st * (S::STAGE_BYTES / 2) + j * 8;
+        const uint16_t *sv = sk + S::TILE_WORDS;
+
+        if (mask) {
+            // ---- scores: per batch, lane computes slot sp = pass sp ^ ppass
+            float sc[NB][PPL][G];
+#pragma unroll
+            for (int bi = 0; bi < NB; ++bi) {
+                float v[NV];
+#pragma unroll
+                for (int sp = 0; sp < RB; ++sp) {
+                    const int tok = (bi * RB + (sp ^ ppass)) * TPW + grp;
+                    const uint4 wv = *reinterpret_cast<const uint4 *>(sk + tok * D);
+                    float2 kf[4];
+                    unpack8<BF16>(wv, kf);
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        float2 acc = __fmul2_rn(q2[g][0], kf[0]);
+                        acc = __ffma2_rn(q2[g][1], kf[1], acc);
+                        acc = __ffma2_rn(q2[g][2], kf[2], acc);
+                        acc = __ffma2_rn(q2[g][3], kf[3], acc);
+                        v[sp * G + g] = acc.x + acc.y;
+                    }
+                }
+                // sum over the token's lanes; halving steps keep the lower slots
+#pragma unroll
+                for (int l = 0; l < S::LEVELS; ++l) {
+                    if (l < HALV) {
+                        const int half = (RB >> (l + 1)) * G;
+#pragma unroll
+                        for (int k = 0; k < NV / 2; ++k)
+                            if (k < half) v[k] += __shfl_xor_sync(0xffffffffu, v[k + half], 1 << l);
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < PPL * G; ++k) v[k] += __shfl_xor_sync(0xffffffffu, v[k], 1 << l);
+                    }
+                }
+#pragma unroll
+                for (int sp = 0; sp < PPL; ++sp) {
+                    const int tok = (bi * RB + ppass + sp) * TPW + grp;
+                    const bool valid = (mask >> tok) & 1u;
+#pragma unroll
+                    for (int g = 0; g < G; ++g) sc[bi][sp][g] = valid ? v[sp * G + g] : -INFINITY;
+                }
+            }
+            // ---- tile max per head over the distinct lanes (pass bits and token groups)
+            float mt[G];
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                mt[g] = sc[0][0][g];
+#pragma unroll
+                for (int bi = 0; bi < NB; ++bi)
+#pragma unroll
+                    for (int sp = 0; sp < PPL; ++sp) mt[g] = fmaxf(mt[g], sc[bi][sp][g]);
+            }
+#pragma unroll
+            for (int l = 0; l < 5; ++l) {
+                if (l >= HALV && l < S::LEVELS) continue;  // copies hold equal values
+#pragma unroll
+                for (int g = 0; g < G; ++g) mt[g] = fmaxf(mt[g], __shfl_xor_sync(0xffffffffu, mt[g], 1 << l));
+            }
+            float alpha[G];
+            bool moved = false;
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const float mn = fmaxf(m_run[g], mt[g]);
+                alpha[g] = (mn == m_run[g]) ? 1.0f : ex2(m_run[g] - mn);
                 moved |= (mn != m_run[g]);
                 m_run[g] = mn;
-                if (g == hl) m_me = mn, a_me = alpha[g];
             }
-            float psum = 0.0f;
+            // ---- probabilities: one exp2 per score; publish (p, p) pairs
 #pragma unroll
-            for (int it = 0; it < ITERS; ++it) {
-                const float pv = (sc[it] == -INFINITY) ? 0.0f : exp2f(sc[it] - m_me);
-                sc[it] = pv;
-                psum += pv;
+            for (int g = 0; g < G; ++g) {
+                float ps = 0.0f;
+#pragma unroll
+                for (int bi = 0; bi < NB; ++bi)
+#pragma unroll
+                    for (int sp = 0; sp < PPL; ++sp) {
+                        const float x = sc[bi][sp][g];
+                        const float pv = (x == -INFINITY) ? 0.0f : ex2(x - m_run[g]);
+                        sc[bi][sp][g] = pv;
+                        ps += pv;
+                    }
+                l_run[g] = l_run[g] * alpha[g] + ps;
             }
-            l_run = l_run * a_me + psum;
             if (moved) {
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
                     const float2 a2 = make_float2(alpha[g], alpha[g]);
 #pragma unroll
-                    for (int k = 0; k < DPL / 2; ++k) o2[g][k] = __fmul2_rn(o2[g][k], a2);
+                    for (int k = 0; k < 4; ++k) o2[g][k] = __fmul2_rn(o2[g][k], a2);
                 }
             }
-            if ((j & ((1 << S::HSHIFT) - 1)) == 0) {
+            if (primary) {
 #pragma unroll
-                for (int it = 0; it < ITERS; ++it) pw[(it * TPW + grp) * G + hl] = sc[it];
+                for (int bi = 0; bi < NB; ++bi)
+#pragma unroll
+                    for (int sp = 0; sp < PPL; ++sp) {
+                        const int tok = (bi * RB + ppass + sp) * TPW + grp;
+#pragma unroll
+                        for (int g = 0; g < G; g += 2) {
+                            const float a = sc[bi][sp][g];
+                            const float b = (g + 1 < G) ? sc[bi][sp][g + 1] : 0.0f;
+                            if (g + 1 < G)
+                                *reinterpret_cast<float4 *>(pw + tok * G + g) = make_float4(a, a, b, b);
+                            else
+                                pw[tok * G + g] = make_float2(a, a);
+                        }
+                    }
             }
             __syncwarp();
             // ---- P.V
@@ -337,193 +552,182 @@ __global__ void __launch_bounds__(NW * 32, 3) decode_kernel(const Params p)
             for (int it = 0; it < ITERS; ++it) {
                 const int tok = it * TPW + grp;
                 if (!((mask >> tok) & 1u)) continue;
-                float pg[G];
+                float2 pp[G];
 #pragma unroll
                 for (int g = 0; g < G; g += 2) {
                     if (g + 1 < G) {
-                        const float2 t2 = *reinterpret_cast<const float2 *>(pw + tok * G + g);
-                        pg[g] = t2.x, pg[g + 1] = t2.y;
+                        const float4 t4 = *reinterpret_cast<const float4 *>(pw + tok * G + g);
+                        pp[g] = make_float2(t4.x, t4.y);
+                        pp[g + 1] = make_float2(t4.z, t4.w);
                     } else {
-                        pg[g] = pw[tok * G + g];
+                        pp[g] = pw[tok * G + g];
                     }
                 }
-                const uint16_t *vrow = sv + tok * D;
+                const uint4 wv = *reinterpret_cast<const uint4 *>(sv + tok * D);
+                float2 vf[4];
+                unpack8<BF16>(wv, vf);
 #pragma unroll
-                for (int c = 0; c < CH; ++c) {
-                    const uint4 w = *reinterpret_cast<const uint4 *>(vrow + (j + c * LPT) * 8);
-                    float2 vf[4];
-                    unpack8<BF16>(w, vf);
+                for (int g = 0; g < G; ++g)
 #pragma unroll
-                    for (int g = 0; g < G; ++g) {
-                        const float2 pp = make_float2(pg[g], pg[g]);
+                    for (int e = 0; e < 4; ++e) o2[g][e] = __ffma2_rn(pp[g], vf[e], o2[g][e]);
+            }
+        }
+        __syncwarp();  // stage and P buffer are free again
+        if (prod.t < t_end) {
+            if (lane == 0) {
+                fence_proxy_async_smem();
+                issue(prod, pseq % NST, pf_blk, pf_ctx);
+            }
+            advance(prod);
+            ++pseq;
+            if (lane == 0 && prod.t < t_end) fetch(prod, pf_blk, pf_ctx);
+        }
+
+        // ---- end of this warp's segment of the (r, h) context
+        if (cons.ti == cons.nt - 1 || cons.t == t_end - 1) {
+            const int r = cons.r, h = cons.h, nt = cons.nt;
+            // softmax sums per head over the distinct lanes
+            float lh[G];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) o2[g][c * 4 + e] = __ffma2_rn(pp, vf[e], o2[g][c * 4 + e]);
-                    }
+            for (int g = 0; g < G; ++g) lh[g] = l_run[g];
+#pragma unroll
+            for (int l = 0; l < 5; ++l) {
+                if (l >= HALV && l < S::LEVELS) continue;
+#pragma unroll
+                for (int g = 0; g < G; ++g) lh[g] += __shfl_xor_sync(0xffffffffu, lh[g], 1 << l);
+            }
+            // outputs: sum over the TPW token groups (lane bits LPT, 2 LPT, ...)
+            float2 ov[S::NO];
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) ov[g * 4 + k] = o2[g][k];
+            transposed_reduce<S::NO, S::OLEV>(ov, lane, LPT, 32,
+                                              [](float2 a, float2 b) { return make_float2(a.x + b.x, a.y + b.y); });
+            const int obase = halving_base<S::NO, S::OLEV>(lane, LPT);
+            // the warps covering this context's global tiles [A, A + nt)
+            const int A = s_pref[r] + h * nt;
+            const int w_first = static_cast<int>(((static_cast<int64_t>(A) + 1) * W - 1) / total);
+            const int w_last = static_cast<int>(((static_cast<int64_t>(A) + nt) * W - 1) / total);
+            float *out_rh = p.out + (static_cast<size_t>(r) * p.Hq + static_cast<size_t>(h) * G) * D;
+            const bool whole = (w_first == w_last);
+            const int rhidx = r * Hkv + h;
+            float *slot = p.part + static_cast<size_t>(w + rhidx) * G * (D + 2);
+#pragma unroll
+            for (int x = 0; x < S::OVPL; ++x) {
+                const int k = obase + x;
+                const int g = k / 4, dim = j * 8 + (k % 4) * 2;
+                float lg = 0.0f;
+#pragma unroll
+                for (int gg = 0; gg < G; ++gg)
+                    if (gg == g) lg = lh[gg];
+                if (whole) {
+                    const float inv = lg > 0.0f ? 1.0f / lg : 0.0f;
+                    *reinterpret_cast<float2 *>(out_rh + g * D + dim) = make_float2(ov[x].x * inv, ov[x].y * inv);
+                } else {
+                    *reinterpret_cast<float2 *>(slot + g * D + dim) = ov[x];
+                }
+            }
+            if (!whole) {
+                if (lane < G) {
+                    float mg = 0.0f, lg = 0.0f;
+#pragma unroll
+                    for (int gg = 0; gg < G; ++gg)
+                        if (gg == lane) mg = m_run[gg], lg = lh[gg];
+                    slot[G * D + lane * 2 + 0] = mg;
+                    slot[G * D + lane * 2 + 1] = lg;
+                }
+                __threadfence();
+                __syncwarp();
+                int last = 0;
+                if (lane == 0) last = atomicAdd(&p.counters[rhidx], 1) == (w_last - w_first);
+                last = __shfl_sync(0xffffffffu, last, 0);
+                if (last) {
+                    __threadfence();
+                    combine<D, G>(p, rhidx, w_first, w_last, lane, out_rh);
+                    if (lane == 0) p.counters[rhidx] = 0;
                 }
             }
         }
-        __syncwarp();
-        if (i + NST < nt_w && lane == 0) {
-            fence_proxy_async_smem();
-            issue(i + NST);
-        }
-        __syncwarp();
+        advance(cons);
     }
+}
 
-    // ---- merge the token groups' sums, then the warps, in shared memory
-#pragma unroll
-    for (int off = LPT; off < 32; off <<= 1) l_run += __shfl_xor_sync(0xffffffffu, l_run, off);
-    __syncthreads();  // every warp is done with its stages
-    float *cm_o = reinterpret_cast<float *>(smem);  // [NW][TPW][G][D], aliases the stages
-    if (lane == 0)
-#pragma unroll
-        for (int g = 0; g < G; ++g) cm_m[warp * G + g] = m_run[g];
-    if (grp == 0 && (j & ((1 << S::HSHIFT) - 1)) == 0) cm_l[warp * G + hl] = l_run;
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-        for (int c = 0; c < CH; ++c) {
-            float *dst = cm_o + ((warp * TPW + grp) * G + g) * D + (j + c * LPT) * 8;
-            reinterpret_cast<float4 *>(dst)[0] =
-                make_float4(o2[g][c * 4].x, o2[g][c * 4].y, o2[g][c * 4 + 1].x, o2[g][c * 4 + 1].y);
-            reinterpret_cast<float4 *>(dst)[1] =
-                make_float4(o2[g][c * 4 + 2].x, o2[g][c * 4 + 2].y, o2[g][c * 4 + 3].x, o2[g][c * 4 + 3].y);
-        }
-    __syncthreads();
-
-    const size_t rh = static_cast<size_t>(r) * p.Hkv + h;
-    for (int idx = tid; idx < G * D; idx += NW * 32) {
-        const int g = idx / D, d = idx % D;
-        float Mx = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) Mx = fmaxf(Mx, cm_m[w * G + g]);
-        float L = 0.0f, O = 0.0f;
-        if (Mx != -INFINITY) {
-#pragma unroll
-            for (int w = 0; w < NW; ++w) {
-                const float mw = cm_m[w * G + g];
-                if (mw == -INFINITY) continue;
-                const float f = exp2f(mw - Mx);
-                L += cm_l[w * G + g] * f;
-                float ow = 0.0f;
-#pragma unroll
-                for (int t = 0; t < TPW; ++t) ow += cm_o[((w * TPW + t) * G + g) * D + d];
-                O += ow * f;
-            }
-        }
-        if (nsplit == 1) {
-            out_rh[idx] = L > 0.0f ? O / L : 0.0f;
-        } else {
-            p.ws_o[((rh * p.max_splits + split) * G + g) * D + d] = O;
-            if (d == 0) {
-                p.ws_ml[((rh * p.max_splits + split) * G + g) * 2 + 0] = Mx;
-                p.ws_ml[((rh * p.max_splits + split) * G + g) * 2 + 1] = L;
-            }
-        }
+// ------------------------------------------------------------------- host
+static int sm_count(int dev)
+{
+    static int cache[64] = {0};
+    if (dev < 0 || dev >= 64) return 0;
+    if (!cache[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        cache[dev] = n;
     }
-    if (nsplit == 1) return;
-
-    // ---- split-K: the last split of (r, h) to finish combines all partials
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) *sflag = atomicAdd(&p.counters[rh], 1) == nsplit - 1;
-    __syncthreads();
-    if (!*sflag) return;
-    __threadfence();
-    float *wts = reinterpret_cast<float *>(smem);  // [nsplit][G] weights, then [G] total
-    float *tot = wts + kMaxSplits * G;
-    const float *ml = p.ws_ml + rh * p.max_splits * G * 2;
-    if (tid < G) {
-        float Mx = -INFINITY;
-        for (int s2 = 0; s2 < nsplit; ++s2) Mx = fmaxf(Mx, __ldcg(ml + (s2 * G + tid) * 2));
-        float L = 0.0f;
-        for (int s2 = 0; s2 < nsplit; ++s2) {
-            const float ms = __ldcg(ml + (s2 * G + tid) * 2);
-            const float f = (ms == -INFINITY) ? 0.0f : exp2f(ms - Mx);
-            wts[s2 * G + tid] = f;
-            L += __ldcg(ml + (s2 * G + tid) * 2 + 1) * f;
-        }
-        tot[tid] = L > 0.0f ? 1.0f / L : 0.0f;
-    }
-    __syncthreads();
-    const float *po = p.ws_o + rh * p.max_splits * G * D;
-    for (int idx = tid; idx < G * D; idx += NW * 32) {
-        const int g = idx / D;
-        float O = 0.0f;
-        for (int s2 = 0; s2 < nsplit; ++s2) O += __ldcg(po + static_cast<size_t>(s2) * G * D + idx) * wts[s2 * G + g];
-        out_rh[idx] = O * tot[g];
-    }
-    if (tid == 0) p.counters[rh] = 0;
+    return cache[dev];
 }
 
 template <int D, int G>
-static int launch(const Params &p, bool bf16, int B, cudaStream_t s)
+static int warps_per_cta() { return Shape<D, G>::NW; }
+
+static int nw_for(int D, int G)
 {
-    const size_t smem = Smem<D, G>::total(p.chunk_blocks);
+#define KVP_NW(d, g) \
+    if (D == d && G == g) return warps_per_cta<d, g>();
+    KVP_NW(64, 1) KVP_NW(64, 2) KVP_NW(64, 4) KVP_NW(64, 8)
+    KVP_NW(128, 1) KVP_NW(128, 2) KVP_NW(128, 4) KVP_NW(128, 8)
+    KVP_NW(256, 1) KVP_NW(256, 2) KVP_NW(256, 4) KVP_NW(256, 8)
+#undef KVP_NW
+    return 0;
+}
+
+struct Layout {
+    int warps_total, min_tiles;
+    size_t counters, part, total;
+};
+
+static int plan(const kvp_pool *pool, int G, int Hkv, int B, int max_ctx, int split_req, Layout *L)
+{
+    if (split_req < 0 || split_req % TT)
+        return set_error(KVP_EINVAL, "split_tokens %d must be 0 or a positive multiple of %d", split_req, TT);
+    if (B < 0 || B > kMaxBatch) return set_error(KVP_EUNSUPPORTED, "B %d outside [0, %d]", B, kMaxBatch);
+    if (max_ctx < 0) return set_error(KVP_EINVAL, "max_ctx_len must be >= 0");
+    const int nw = nw_for(pool->cfg.head_dim, G);
+    if (!nw) return set_error(KVP_EUNSUPPORTED, "decode: head_dim %d with GQA group %d not built", pool->cfg.head_dim, G);
+    const int sms = sm_count(pool->cfg.device);
+    if (!sms) return set_error(KVP_ECUDA, "cannot query the SM count of device %d", pool->cfg.device);
+    L->warps_total = sms * nw;
+    L->min_tiles = split_req > 0 ? split_req / TT : kAutoMinTiles;
+    const size_t rh = static_cast<size_t>(B) * Hkv;
+    const size_t slot = static_cast<size_t>(G) * (pool->cfg.head_dim + 2) * 4;
+    L->counters = 0;
+    L->part = align_up(rh * 4, 256);
+    L->total = align_up(L->part + (L->warps_total + rh) * slot, 256);
+    return KVP_OK;
+}
+
+template <int D, int G>
+static int launch(const Params &p, bool bf16, int blocks, cudaStream_t s)
+{
+    const size_t smem = Smem<D, G>::total(p.B);
     if (smem > 227 * 1024) return set_error(KVP_EUNSUPPORTED, "decode: %zu bytes of shared memory", smem);
     auto kern = bf16 ? decode_kernel<D, G, true> : decode_kernel<D, G, false>;
     int rc = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)),
                         "decode smem attribute");
     if (rc) return rc;
-    dim3 grid(p.max_splits, p.Hkv, B);
-    kern<<<grid, NW * 32, smem, s>>>(p);
+    kern<<<blocks, Shape<D, G>::NW * 32, smem, s>>>(p);
     return check_cuda(cudaGetLastError(), "decode launch");
 }
 
 template <int D>
-static int launch_g(const Params &p, bool bf16, int B, int G, cudaStream_t s)
+static int launch_g(const Params &p, bool bf16, int blocks, int G, cudaStream_t s)
 {
     switch (G) {
-    case 1: return launch<D, 1>(p, bf16, B, s);
-    case 2: return launch<D, 2>(p, bf16, B, s);
-    case 4: return launch<D, 4>(p, bf16, B, s);
-    case 8: return launch<D, 8>(p, bf16, B, s);
+    case 1: return launch<D, 1>(p, bf16, blocks, s);
+    case 2: return launch<D, 2>(p, bf16, blocks, s);
+    case 4: return launch<D, 4>(p, bf16, blocks, s);
+    case 8: return launch<D, 8>(p, bf16, blocks, s);
     default: return set_error(KVP_EUNSUPPORTED, "decode: GQA group %d not built (1, 2, 4, 8)", G);
     }
-}
-
-// Split size: multiples of max(16, block_size); ~256 keys, smaller when the
-// batch is too small to fill 4 CTAs per SM, larger when a context would need
-// more than kMaxSplits splits.
-static int choose_split(int bs, int B, int Hkv, int max_ctx, int requested)
-{
-    const int unit = bs > TT ? bs : TT;
-    if (requested > 0) return requested;
-    if (max_ctx <= 0) return unit;
-    auto up = [&](long long x) { return static_cast<int>((x + unit - 1) / unit * unit); };
-    int split = up(256);
-    const long long units = static_cast<long long>(B) * Hkv;
-    const long long target = 4LL * 148;
-    if (units * ((max_ctx + split - 1) / split) < target) {
-        split = up((static_cast<long long>(max_ctx) * units + target - 1) / target);
-        if (split < unit) split = unit;
-    }
-    if ((max_ctx + split - 1) / split > kMaxSplits) split = up((max_ctx + kMaxSplits - 1) / kMaxSplits);
-    return split;
-}
-
-struct Layout {
-    int split, max_splits;
-    size_t counters, ml, o, total;
-};
-
-static int plan(const kvp_pool *pool, int G, int Hkv, int B, int max_ctx, int split_req, Layout *L)
-{
-    const int bs = pool->cfg.block_size;
-    const int unit = bs > TT ? bs : TT;
-    if (split_req < 0 || (split_req > 0 && split_req % unit))
-        return set_error(KVP_EINVAL, "split_tokens %d must be 0 or a multiple of %d", split_req, unit);
-    if (B < 0 || max_ctx < 0) return set_error(KVP_EINVAL, "B and max_ctx_len must be >= 0");
-    L->split = choose_split(bs, B, Hkv, max_ctx, split_req);
-    L->max_splits = max_ctx > 0 ? (max_ctx + L->split - 1) / L->split : 1;
-    if (L->max_splits > kMaxSplits)
-        return set_error(KVP_EINVAL, "split_tokens %d gives %d splits (max %d)", L->split, L->max_splits, kMaxSplits);
-    const size_t rh = static_cast<size_t>(B) * Hkv;
-    L->counters = 0;
-    L->ml = align_up(rh * 4, 256);
-    L->o = align_up(L->ml + rh * L->max_splits * G * 2 * 4, 256);
-    L->total = align_up(L->o + rh * L->max_splits * G * pool->cfg.head_dim * 4, 256);
-    return KVP_OK;
 }
 
 }  // namespace dec
@@ -552,7 +756,6 @@ extern "C" int paged_decode_attention(kvp_pool *pool, int layer, const kvp_attn_
     int Hq, Hkv, G;
     if ((rc = resolve_attn(pool, attn, &Hq, &Hkv, &G))) return rc;
     if (B == 0) return KVP_OK;
-    if (B < 0 || B > 65535) return set_error(KVP_EINVAL, "B %d outside [0, 65535]", B);
     if (max_blocks_per_seq <= 0) return set_error(KVP_EINVAL, "max_blocks_per_seq must be > 0");
     if (!q || !block_tables || !ctx_lens || !out || !workspace)
         return set_error(KVP_EINVAL, "paged_decode_attention: a required pointer is NULL");
@@ -561,29 +764,27 @@ extern "C" int paged_decode_attention(kvp_pool *pool, int layer, const kvp_attn_
     if (reinterpret_cast<uintptr_t>(workspace) & 255) return set_error(KVP_EINVAL, "workspace must be 256-byte aligned");
     dec::Layout L;
     if ((rc = dec::plan(pool, G, Hkv, B, max_ctx_len, split_tokens, &L))) return rc;
-    if (ws_bytes < L.total)
-        return set_error(KVP_EINVAL, "workspace of %zu bytes, %zu needed", ws_bytes, L.total);
+    if (ws_bytes < L.total) return set_error(KVP_EINVAL, "workspace of %zu bytes, %zu needed", ws_bytes, L.total);
     dec::Params p;
     p.kp = pool->k_base + pool->layer_words * layer;
     p.vp = pool->v_base + pool->layer_words * layer;
     p.q = q, p.bt = block_tables, p.ctx = ctx_lens, p.out = out;
     unsigned char *ws = static_cast<unsigned char *>(workspace);
     p.counters = reinterpret_cast<int *>(ws + L.counters);
-    p.ws_ml = reinterpret_cast<float *>(ws + L.ml);
-    p.ws_o = reinterpret_cast<float *>(ws + L.o);
+    p.part = reinterpret_cast<float *>(ws + L.part);
     p.status = pool->status;
-    p.Hq = Hq, p.Hkv = Hkv, p.mbps = max_blocks_per_seq, p.bs = pool->cfg.block_size;
+    p.B = B, p.Hq = Hq, p.Hkv = Hkv, p.mbps = max_blocks_per_seq, p.bs = pool->cfg.block_size;
     p.num_blocks = pool->cfg.num_blocks, p.max_ctx = max_ctx_len, p.max_seq_len = pool->cfg.max_seq_len;
-    p.split = L.split, p.max_splits = L.max_splits;
-    p.chunk_blocks = L.split / p.bs + 1;
+    p.warps_total = L.warps_total, p.min_tiles = L.min_tiles;
     const double scale = static_cast<double>(static_cast<float>(1.0 / sqrt(static_cast<double>(pool->cfg.head_dim))));
     p.qscale = static_cast<float>(scale * 1.4426950408889634);  // log2(e): softmax via exp2
     const bool bf16 = pool->cfg.kv_dtype == KVP_BF16;
+    const int blocks = L.warps_total / dec::nw_for(pool->cfg.head_dim, G);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     switch (pool->cfg.head_dim) {
-    case 64: return dec::launch_g<64>(p, bf16, B, G, s);
-    case 128: return dec::launch_g<128>(p, bf16, B, G, s);
-    case 256: return dec::launch_g<256>(p, bf16, B, G, s);
+    case 64: return dec::launch_g<64>(p, bf16, blocks, G, s);
+    case 128: return dec::launch_g<128>(p, bf16, blocks, G, s);
+    case 256: return dec::launch_g<256>(p, bf16, blocks, G, s);
     default: return set_error(KVP_EUNSUPPORTED, "head_dim %d", pool->cfg.head_dim);
     }
 }

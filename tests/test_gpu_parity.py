@@ -87,10 +87,9 @@ def test_append_and_decode_small(orc, dev, name):
     q_ref, pk, pv = _check_append(orc, run)
     st, ref = oracle_decode(orc, wl, q_ref, pk, pv)
     assert st == 0
-    unit = max(16, wl.spec.bs)
-    mx = int(wl.ctx.max())
-    finest = unit * max(1, -(-mx // (unit * 100)))  # the smallest split giving <= 100 splits
-    for split in (0, finest, 4 * finest):
+    # split_tokens = the fewest keys a warp takes: 16 spreads contexts over
+    # many warps (many partials), a huge value puts everything on one warp
+    for split in (0, 16, 96, 1 << 20):
         out = run.decode(split_tokens=split)
         run.pool.sync_status()
         assert_close(out.cpu().numpy(), ref, f"{name} split={split}")
@@ -116,9 +115,9 @@ def test_split_invariance_and_single_split_identity(orc, dev):
     wl = make_workload(SMALL["gqa8-long"])
     run = GpuRun(wl, dev)
     run.append()
-    one = run.decode(split_tokens=4112)  # one split covers every context here
+    one = run.decode(split_tokens=1 << 20)  # one warp takes every context: no partials
     run.pool.sync_status()
-    for split in (48, 96, 256, 0):
+    for split in (16, 48, 256, 0):
         out = run.decode(split_tokens=split)
         run.pool.sync_status()
         assert_close(out.cpu().numpy(), one.cpu().numpy(), f"split {split} vs 1")

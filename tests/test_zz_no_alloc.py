@@ -44,12 +44,12 @@ def test_noalloc_refuses_calls_above_its_fixed_size():
     from gpu_harness import GpuRun
     from workloads import Segment, Spec, make_workload
 
-    spec = Spec(name="noalloc-big", Hq=8, Hkv=2, D=128, bs=16, kv_dtype="f16", theta=0.0,
+    spec = Spec(name="noalloc-big", Hq=32, Hkv=8, D=128, bs=16, kv_dtype="f16", theta=0.0,
                 segments=(Segment(q_len=1, fixed=(40,)),), seed_offset=301)
     wl = make_workload(spec)
     run = GpuRun(wl, torch.device("cuda", 0))
     q, bt, ctx, mx = run.decode_inputs()
-    B = 4096  # many sequences with long contexts need far more than 16 MiB
+    B = 2048  # partials of 2048 sequences x 8 kv heads need far more than 16 MiB
     big = K.decode_workspace_size(run.pool, run.attn, B, 20000)
     assert big > K.NOALLOC_SCRATCH_BYTES
     qq = q.expand(B, -1, -1).contiguous()
