@@ -35,6 +35,8 @@
 //    counter, so no second launch is needed.
 #include <math.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace kvp {
@@ -45,6 +47,7 @@ constexpr int NST = 2;             // stages per warp
 constexpr int kMaxBatch = 2048;    // sequences per call (per-CTA prefix in shared memory)
 constexpr int kAutoMinTiles = 2;   // default minimum tiles per warp
 constexpr int kStageBudget = 200 * 1024;
+constexpr float kLazy = 8.0f;   // log2 headroom before the reference max must move
 
 constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
 constexpr int cmin(int a, int b) { return a < b ? a : b; }
@@ -96,7 +99,7 @@ struct Smem {
     using S = Shape<D, G>;
     static constexpr size_t stages = 0;
     static constexpr size_t bars = static_cast<size_t>(S::NW) * NST * S::STAGE_BYTES;
-    static constexpr size_t masks = bars + S::NW * NST * 8;
+    static constexpr size_t masks = bars + S::NW * NST * 2 * 8;
     static constexpr size_t pbuf = align_up(masks + S::NW * NST * 4, 16);
     static constexpr size_t tiles = pbuf + S::NW * TT * G * 8;  // [B] tiles per sequence
     __host__ __device__ static size_t pref(int B) { return align_up(tiles + 4 * static_cast<size_t>(B), 16); }  // [B + 1]
@@ -287,8 +290,9 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
     const int t_end = static_cast<int>(static_cast<int64_t>(w + 1) * total / W);
     if (t_begin >= t_end) return;  // no CTA-wide barrier follows
 
-    const uint32_t bar0 = smem_addr(&bars[warp * NST]);
-    if (lane < NST) mbar_init(bar0 + lane * 8, 1);
+    // barriers: [warp][stage][K, V] "tile half landed"
+    const uint32_t kbar0 = smem_addr(&bars[warp * NST * 2]);
+    if (lane < 2 * NST) mbar_init(kbar0 + lane * 8, 1);
     mbar_init_fence();
     __syncwarp();
 
@@ -321,80 +325,104 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
     };
 
     uint16_t *wst = stages + static_cast<size_t>(warp) * NST * (S::STAGE_BYTES / 2);
+    int *nvalid = reinterpret_cast<int *>(masks) + warp * NST;
     float2 *pw = pbuf + warp * TT * G;  // (p, p) pairs per (token, head)
     const size_t blk_stride = static_cast<size_t>(Hkv) * p.bs * D;
-    const bool big_blocks = p.bs >= TT;  // one block per tile
+    const bool big_blocks = p.bs >= TT;  // a tile lies inside one block
+    const int ntile = t_end - t_begin;
 
-    // Copies tile c into stage st (lane 0 only). For big blocks the tile's
-    // block id and context length come prefetched (blk, ctx).
-    auto issue = [&](const Cursor &c, int st, int blk, int ctx) {
-        const int tb = c.ti * TT;
-        const uint32_t bar = bar0 + st * 8;
-        uint16_t *dk = wst + st * (S::STAGE_BYTES / 2);
-        uint16_t *dv = dk + S::TILE_WORDS;
-        const size_t head_off = static_cast<size_t>(c.h) * p.bs * D;
-        uint32_t mask = 0;
-        if (big_blocks) {
+    // Copy descriptors of 32 consecutive tiles, one per lane: the element
+    // offset of the tile's K (and V) run in the layer pool and its number of
+    // valid tokens (0: block id outside the pool).
+    int64_t d_off = 0;
+    int d_nv = 0, dbase = 0;
+    auto load_desc = [&](int base) {
+        dbase = base;
+        d_off = 0;
+        d_nv = 0;
+        const int i = base + lane;
+        if (big_blocks && i < ntile) {
+            Cursor c;
+            locate(t_begin + i, c);
+            const int ctx = p.ctx[c.r];
+            const int tb = c.ti * TT;
+            const int blk = p.bt[static_cast<size_t>(c.r) * p.mbps + tb / p.bs];
             if (blk >= 0 && blk < p.num_blocks) {
-                mask = (1u << min(TT, ctx - tb)) - 1u;
-                const size_t off = blk * blk_stride + head_off + static_cast<size_t>(tb % p.bs) * D;
-                mbar_arrive_expect_tx(bar, S::STAGE_BYTES);
-                bulk_g2s(smem_addr(dk), p.kp + off, S::TILE_WORDS * 2, bar);
-                bulk_g2s(smem_addr(dv), p.vp + off, S::TILE_WORDS * 2, bar);
+                d_off = static_cast<int64_t>(blk) * blk_stride + static_cast<int64_t>(c.h) * p.bs * D +
+                        static_cast<int64_t>(tb % p.bs) * D;
+                d_nv = min(TT, ctx - tb);
             } else {
                 report(p.status, KVP_ERANGE, c.r);
-                mbar_arrive(bar);
+            }
+        }
+    };
+    // Small blocks (a tile spans several): the issuing lane walks the blocks.
+    auto issue_small = [&](int i, int half, int st) {
+        Cursor c;
+        locate(t_begin + i, c);
+        const int ctx = p.ctx[c.r];
+        const int tb = c.ti * TT;
+        const int32_t *btr = p.bt + static_cast<size_t>(c.r) * p.mbps;
+        const uint32_t bar = kbar0 + (st * 2 + half) * 8;
+        uint16_t *dst = wst + st * (S::STAGE_BYTES / 2) + half * S::TILE_WORDS;
+        const uint16_t *src = half ? p.vp : p.kp;
+        uint32_t bytes = 0;
+        int nv = 0;
+        for (int t = 0; t < TT && tb + t < ctx; t += p.bs) {
+            const int b = btr[(tb + t) / p.bs];
+            if (b >= 0 && b < p.num_blocks) {
+                bytes += p.bs * D * 2;
+                nv = t + min(p.bs, ctx - tb - t);
+            } else {
+                report(p.status, KVP_ERANGE, c.r);
+                break;  // tokens up to the bad block only
+            }
+        }
+        if (bytes) {
+            mbar_arrive_expect_tx(bar, bytes);
+            for (int t = 0; t < nv; t += p.bs) {
+                const int b = btr[(tb + t) / p.bs];
+                bulk_g2s(smem_addr(dst + t * D), src + b * blk_stride + static_cast<size_t>(c.h) * p.bs * D,
+                         p.bs * D * 2, bar);
             }
         } else {
-            const int32_t *btr = p.bt + static_cast<size_t>(c.r) * p.mbps;
-            uint32_t bytes = 0;
-            for (int t = 0; t < TT && tb + t < ctx; t += p.bs) {
-                const int b = btr[(tb + t) / p.bs];
-                if (b >= 0 && b < p.num_blocks) {
-                    bytes += 2 * p.bs * D * 2;
-                    mask |= ((1u << min(p.bs, ctx - tb - t)) - 1u) << t;
-                } else {
-                    report(p.status, KVP_ERANGE, c.r);
-                }
-            }
-            if (bytes) {
-                mbar_arrive_expect_tx(bar, bytes);
-                for (int t = 0; t < TT && tb + t < ctx; t += p.bs) {
-                    const int b = btr[(tb + t) / p.bs];
-                    if (b >= 0 && b < p.num_blocks) {
-                        const size_t off = b * blk_stride + head_off;
-                        bulk_g2s(smem_addr(dk + t * D), p.kp + off, p.bs * D * 2, bar);
-                        bulk_g2s(smem_addr(dv + t * D), p.vp + off, p.bs * D * 2, bar);
-                    }
-                }
-            } else {
-                mbar_arrive(bar);
-            }
+            mbar_arrive(bar);
         }
-        masks[warp * NST + st] = mask;
+        if (half == 0) nvalid[st] = nv;
     };
-    // block id and context length of tile c (lane 0; plain loads, used one issue later)
-    auto fetch = [&](const Cursor &c, int &blk, int &ctx) {
-        ctx = p.ctx[c.r];
-        blk = big_blocks ? p.bt[static_cast<size_t>(c.r) * p.mbps + (c.ti * TT) / p.bs] : 0;
+    // Issues half (0: K, 1: V) of tile i (warp-relative) into stage st.
+    auto issue = [&](int i, int half, int st) {
+        if (big_blocks) {
+            if (i - dbase >= 32) load_desc(i);
+            const int64_t off = __shfl_sync(0xffffffffu, d_off, i - dbase);
+            const int nv = __shfl_sync(0xffffffffu, d_nv, i - dbase);
+            if (lane == 0) {
+                fence_proxy_async_smem();
+                const uint32_t bar = kbar0 + (st * 2 + half) * 8;
+                if (nv > 0) {
+                    mbar_arrive_expect_tx(bar, S::TILE_WORDS * 2);
+                    bulk_g2s(smem_addr(wst + st * (S::STAGE_BYTES / 2) + half * S::TILE_WORDS),
+                             (half ? p.vp : p.kp) + off, S::TILE_WORDS * 2, bar);
+                } else {
+                    mbar_arrive(bar);
+                }
+                if (half == 0) nvalid[st] = nv;
+            }
+        } else if (lane == 0) {
+            fence_proxy_async_smem();
+            issue_small(i, half, st);
+        }
     };
 
-    Cursor prod, cons;
-    locate(t_begin, prod);
-    cons = prod;
-    int pseq = 0;
-    int pf_blk = 0, pf_ctx = 0;  // prefetched for the next tile to issue (lane 0)
-    for (int i = 0; i < NST && prod.t < t_end; ++i) {
-        if (lane == 0) {
-            int blk, ctx;
-            fetch(prod, blk, ctx);
-            issue(prod, i, blk, ctx);
-        }
-        advance(prod);
-        ++pseq;
+    load_desc(0);
+    for (int i = 0; i < NST && i < ntile; ++i) {
+        issue(i, 0, i);
+        issue(i, 1, i);
     }
-    if (lane == 0 && prod.t < t_end) fetch(prod, pf_blk, pf_ctx);
     __syncwarp();
+
+    Cursor cons;
+    locate(t_begin, cons);
 
     // ---- per-lane state
     const int grp = lane / LPT, j = lane % LPT;
@@ -411,8 +439,8 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
     float2 o2[G][4];
     float m_run[G], l_run[G];
 
-    for (int seq = 0; cons.t < t_end; ++seq) {
-        if (cons.t == t_begin || cons.ti == 0) {  // a new context segment starts
+    for (int seq = 0; seq < ntile; ++seq) {
+        if (seq == 0 || cons.ti == 0) {  // a new context segment starts
             const float *qb = p.q + (static_cast<size_t>(cons.r) * p.Hq + static_cast<size_t>(cons.h) * G) * D + j * 8;
 #pragma unroll
             for (int g = 0; g < G; ++g) {
@@ -430,16 +458,18 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
         }
 
         const int st = seq % NST;
-        const bool done = mbar_wait_bounded(bar0 + st * 8, (seq / NST) & 1);
-        if (!__all_sync(0xffffffffu, done)) {
+        const uint32_t par = (seq / NST) & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(kbar0 + st * 16, par))) {
             if (lane == 0) report(p.status, KVP_ETIMEOUT, cons.r);
             return;
         }
-        const uint32_t mask = masks[warp * NST + st];
+        const int nv = nvalid[st];
+        const uint32_t mask = (1u << nv) - 1u;
         const uint16_t *sk = wst + st * (S::STAGE_BYTES / 2) + j * 8;
         const uint16_t *sv = sk + S::TILE_WORDS;
 
-        if (mask) {
+        auto tile_qk = [&](auto full_tag) {
+            constexpr bool FULL = decltype(full_tag)::value;
             // ---- scores: per batch, lane computes slot sp = pass sp ^ ppass
             float sc[NB][PPL][G];
 #pragma unroll
@@ -476,35 +506,53 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
 #pragma unroll
                 for (int sp = 0; sp < PPL; ++sp) {
                     const int tok = (bi * RB + ppass + sp) * TPW + grp;
-                    const bool valid = (mask >> tok) & 1u;
+                    const bool valid = FULL || ((mask >> tok) & 1u);
 #pragma unroll
                     for (int g = 0; g < G; ++g) sc[bi][sp][g] = valid ? v[sp * G + g] : -INFINITY;
                 }
             }
-            // ---- tile max per head over the distinct lanes (pass bits and token groups)
-            float mt[G];
+            // ---- reference max per head. Scores are exponentiated against a
+            // per-head reference m_run that only moves when some score exceeds
+            // it by more than kLazy (log2 units), so p stays below 2^kLazy and
+            // most tiles need no warp-wide max and no rescale.
+            bool above = false;
 #pragma unroll
-            for (int g = 0; g < G; ++g) {
-                mt[g] = sc[0][0][g];
+            for (int g = 0; g < G; ++g)
 #pragma unroll
                 for (int bi = 0; bi < NB; ++bi)
 #pragma unroll
-                    for (int sp = 0; sp < PPL; ++sp) mt[g] = fmaxf(mt[g], sc[bi][sp][g]);
-            }
-#pragma unroll
-            for (int l = 0; l < 5; ++l) {
-                if (l >= HALV && l < S::LEVELS) continue;  // copies hold equal values
-#pragma unroll
-                for (int g = 0; g < G; ++g) mt[g] = fmaxf(mt[g], __shfl_xor_sync(0xffffffffu, mt[g], 1 << l));
-            }
+                    for (int sp = 0; sp < PPL; ++sp) above |= sc[bi][sp][g] > m_run[g] + kLazy;
             float alpha[G];
-            bool moved = false;
 #pragma unroll
-            for (int g = 0; g < G; ++g) {
-                const float mn = fmaxf(m_run[g], mt[g]);
-                alpha[g] = (mn == m_run[g]) ? 1.0f : ex2(m_run[g] - mn);
-                moved |= (mn != m_run[g]);
-                m_run[g] = mn;
+            for (int g = 0; g < G; ++g) alpha[g] = 1.0f;
+            if (__any_sync(0xffffffffu, above)) {
+                float mt[G];
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    mt[g] = sc[0][0][g];
+#pragma unroll
+                    for (int bi = 0; bi < NB; ++bi)
+#pragma unroll
+                        for (int sp = 0; sp < PPL; ++sp) mt[g] = fmaxf(mt[g], sc[bi][sp][g]);
+                }
+#pragma unroll
+                for (int l = 0; l < 5; ++l) {
+                    if (l >= HALV && l < S::LEVELS) continue;  // copies hold equal values
+#pragma unroll
+                    for (int g = 0; g < G; ++g) mt[g] = fmaxf(mt[g], __shfl_xor_sync(0xffffffffu, mt[g], 1 << l));
+                }
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const float mn = fmaxf(m_run[g], mt[g]);
+                    alpha[g] = (mn == m_run[g]) ? 1.0f : ex2(m_run[g] - mn);
+                    m_run[g] = mn;
+                }
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const float2 a2 = make_float2(alpha[g], alpha[g]);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) o2[g][k] = __fmul2_rn(o2[g][k], a2);
+                }
             }
             // ---- probabilities: one exp2 per score; publish (p, p) pairs
 #pragma unroll
@@ -515,19 +563,11 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
 #pragma unroll
                     for (int sp = 0; sp < PPL; ++sp) {
                         const float x = sc[bi][sp][g];
-                        const float pv = (x == -INFINITY) ? 0.0f : ex2(x - m_run[g]);
+                        const float pv = (!FULL && x == -INFINITY) ? 0.0f : ex2(x - m_run[g]);
                         sc[bi][sp][g] = pv;
                         ps += pv;
                     }
                 l_run[g] = l_run[g] * alpha[g] + ps;
-            }
-            if (moved) {
-#pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    const float2 a2 = make_float2(alpha[g], alpha[g]);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) o2[g][k] = __fmul2_rn(o2[g][k], a2);
-                }
             }
             if (primary) {
 #pragma unroll
@@ -546,12 +586,14 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
                         }
                     }
             }
-            __syncwarp();
+        };
+        auto tile_pv = [&](auto full_tag) {
+            constexpr bool FULL = decltype(full_tag)::value;
             // ---- P.V
 #pragma unroll
             for (int it = 0; it < ITERS; ++it) {
                 const int tok = it * TPW + grp;
-                if (!((mask >> tok) & 1u)) continue;
+                if (!FULL && !((mask >> tok) & 1u)) continue;
                 float2 pp[G];
 #pragma unroll
                 for (int g = 0; g < G; g += 2) {
@@ -571,20 +613,22 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
 #pragma unroll
                     for (int e = 0; e < 4; ++e) o2[g][e] = __ffma2_rn(pp[g], vf[e], o2[g][e]);
             }
+        };
+        if (mask == 0xFFFFu) tile_qk(std::true_type{});
+        else if (nv > 0) tile_qk(std::false_type{});
+        __syncwarp();  // K half and the previous P are free
+        if (seq + NST < ntile) issue(seq + NST, 0, st);
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(kbar0 + st * 16 + 8, par))) {
+            if (lane == 0) report(p.status, KVP_ETIMEOUT, cons.r);
+            return;
         }
-        __syncwarp();  // stage and P buffer are free again
-        if (prod.t < t_end) {
-            if (lane == 0) {
-                fence_proxy_async_smem();
-                issue(prod, pseq % NST, pf_blk, pf_ctx);
-            }
-            advance(prod);
-            ++pseq;
-            if (lane == 0 && prod.t < t_end) fetch(prod, pf_blk, pf_ctx);
-        }
+        if (mask == 0xFFFFu) tile_pv(std::true_type{});
+        else if (nv > 0) tile_pv(std::false_type{});
+        __syncwarp();  // V half and P buffer are free
+        if (seq + NST < ntile) issue(seq + NST, 1, st);
 
         // ---- end of this warp's segment of the (r, h) context
-        if (cons.ti == cons.nt - 1 || cons.t == t_end - 1) {
+        if (cons.ti == cons.nt - 1 || seq == ntile - 1) {
             const int r = cons.r, h = cons.h, nt = cons.nt;
             // softmax sums per head over the distinct lanes
             float lh[G];
