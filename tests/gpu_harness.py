@@ -66,6 +66,26 @@ class GpuRun:
         K.paged_decode_attention(self.pool, sp.layer, self.attn, q, bt, ctx, mx, out, ws, split_tokens)
         return out
 
+    def prefill(self, seqs=None, out=None):
+        """Prefill attention for the given sequences' new tokens (default: all
+        sequences with more than one new token). Returns (out [n, Hq, D], rows)
+        where rows are the new-token indices in order."""
+        wl = self.wl
+        sp = wl.spec
+        seqs = wl.prefill_seqs if seqs is None else np.asarray(seqs)
+        rows = np.concatenate([np.arange(wl.cu_q[r], wl.cu_q[r + 1]) for r in seqs]).astype(np.int64)
+        cu = np.zeros(len(seqs) + 1, dtype=np.int32)
+        cu[1:] = np.cumsum(wl.q_lens[seqs])
+        dev = self.dev
+        q = self.q_out.index_select(0, torch.from_numpy(rows).to(dev)).view(-1, sp.Hq, sp.D).contiguous()
+        s = torch.from_numpy(seqs.astype(np.int64)).to(dev)
+        bt = self.bt.index_select(0, s).contiguous()
+        ctx = self.ctx.index_select(0, s).contiguous()
+        out = torch.full_like(q, float("nan")) if out is None else out
+        K.paged_prefill_attention(self.pool, sp.layer, self.attn, q, torch.from_numpy(cu).to(dev), ctx, bt,
+                                  int(wl.q_lens[seqs].max()), out)
+        return out, rows
+
     def layer_pools(self):
         sp = self.wl.spec
         return (self.pool.k[sp.layer].cpu().numpy().view(np.uint16),
@@ -81,6 +101,17 @@ def oracle_decode(orc, wl, q_out, pk, pv, seqs=None, threads=0):
     st, out, _ = orc.paged_attention(Hq=sp.Hq, Hkv=sp.Hkv, D=sp.D, bs=sp.bs, kv_dtype=sp.kv_dtype, q=q,
                                      q_seq=seqs, q_pos=wl.ctx[seqs] - 1, block_tables=wl.block_tables,
                                      pool_k=pk, pool_v=pv, threads=threads)
+    return st, out
+
+
+def oracle_rows(orc, wl, q_out, pk, pv, rows, threads=0):
+    """Oracle attention for arbitrary new-token rows (query at its position)."""
+    sp = wl.spec
+    rows = np.asarray(rows)
+    st, out, _ = orc.paged_attention(Hq=sp.Hq, Hkv=sp.Hkv, D=sp.D, bs=sp.bs, kv_dtype=sp.kv_dtype,
+                                     q=q_out[rows].reshape(-1, sp.Hq, sp.D), q_seq=wl.tok_req[rows],
+                                     q_pos=wl.positions[rows], block_tables=wl.block_tables, pool_k=pk, pool_v=pv,
+                                     threads=threads)
     return st, out
 
 
