@@ -1,9 +1,11 @@
 """Benchmark of the paged KV cache hot path on B200.
 
 One step = kv_append of every new token (norm, RoPE, 16-bit conversion,
-scatter) followed by paged_decode_attention over every sequence, on the
-Llama-3-8B-shaped batch-32 decode workload (Hq=32, Hkv=8, D=128, bf16 pool,
-block size 16, contexts U[512, 4096]). Inputs are synthetic and seeded.
+scatter) followed by paged_decode_attention over every decoding sequence
+(and, for a mixed workload, paged_prefill_attention over the prefill
+chunks), by default on the Llama-3-8B-shaped batch-32 decode workload
+(Hq=32, Hkv=8, D=128, bf16 pool, block size 16, contexts U[512, 4096]).
+Inputs are synthetic and seeded.
 
 Reports whole-step KV-read throughput (algorithmic K+V bytes of the decode
 pass divided by the step time), the decode kernel against the measured HBM
@@ -55,6 +57,14 @@ def measured_peaks():
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_bf16_tflops():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured burst"
+    except Exception:
+        return 1590.0, "fallback"
 
 
 def sources_sha(paths) -> str:
@@ -126,17 +136,13 @@ class ClockSampler:
 def dist_setup(n_gpus: int):
     import torch
 
-    if n_gpus <= 1 or "RANK" not in os.environ:
+    from paged_kv_cache_321_b200 import replicas
+
+    rank, world, local = replicas.world_from_env()
+    if n_gpus <= 1 or world == 1:
         return 0, 1, None
-    import datetime
-
-    import torch.distributed as dist
-
-    rank, world = int(os.environ["RANK"]), int(os.environ["WORLD_SIZE"])
-    local = int(os.environ.get("LOCAL_RANK", rank))
     torch.cuda.set_device(local)
-    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                            device_id=torch.device("cuda", local))
+    dist = replicas.init("nccl", timeout_s=120, device=torch.device("cuda", local))
     return rank, world, dist
 
 
@@ -227,7 +233,9 @@ def run_ours(args):
     from workloads import SPECS, make_workload
 
     spec = SPECS[args.workload]
-    wl = make_workload(spec, seed_offset=spec.seed_offset + 1000 * rank)  # one independent replica per rank
+    from paged_kv_cache_321_b200 import replicas
+
+    wl = make_workload(spec, seed_offset=replicas.replica_seed_offset(spec.seed_offset, rank))
     sp = wl.spec
     stream = torch.cuda.current_stream()
 
@@ -241,33 +249,79 @@ def run_ours(args):
     q, k, v = g(wl.q), g(wl.k), g(wl.v)
     qn, kn = g(wl.q_norm_w), g(wl.k_norm_w)
     tok_req, positions, bt, ctx = g(wl.tok_req), g(wl.positions), g(wl.block_tables), g(wl.ctx)
-    seqs = wl.decode_seqs
-    assert len(seqs) == wl.S, "the benchmark workload is decode-only"
-    B, T, mx = wl.S, wl.T, int(wl.ctx.max())
+    dseq, pseq = wl.decode_seqs, wl.prefill_seqs
+    T = wl.T
     q_out = torch.empty((T, sp.Hq * sp.D), dtype=torch.float32, device=dev)
+    kv_bytes = wl.kv_read_bytes()  # the decode sequences' K/V
+    # decode inputs: the decode sequences' rows (views when they are all sequences)
+    B = len(dseq)
+    mx = int(wl.ctx[dseq].max(initial=0))
+    sel = lambda t, idx: t if len(idx) == wl.S else t.index_select(0, torch.from_numpy(idx.astype(np.int64)).to(dev))
+    d_bt, d_ctx = sel(bt, dseq).contiguous(), sel(ctx, dseq).contiguous()
+    d_rows = torch.from_numpy(wl.cu_q[dseq].astype(np.int64)).to(dev)
+    d_q = q_out.view(T, sp.Hq, sp.D) if B == T else torch.empty((B, sp.Hq, sp.D), dtype=torch.float32, device=dev)
     out = torch.empty((B, sp.Hq, sp.D), dtype=torch.float32, device=dev)
     ws_n = K.decode_workspace_size(pool, attn, B, mx, args.split_tokens)
     ws = torch.zeros(ws_n // 4 + 64, dtype=torch.float32, device=dev)
-    kv_bytes = wl.kv_read_bytes()
+    # prefill inputs: the chunk sequences' rows
+    prefill_flops = 0
+    if len(pseq):
+        p_rows = np.concatenate([np.arange(wl.cu_q[r], wl.cu_q[r + 1]) for r in pseq]).astype(np.int64)
+        p_rows_t = torch.from_numpy(p_rows).to(dev)
+        p_cu = np.zeros(len(pseq) + 1, dtype=np.int32)
+        p_cu[1:] = np.cumsum(wl.q_lens[pseq])
+        p_cu_t = torch.from_numpy(p_cu).to(dev)
+        p_bt, p_ctx = sel(bt, pseq).contiguous(), sel(ctx, pseq).contiguous()
+        p_q = torch.empty((len(p_rows), sp.Hq, sp.D), dtype=torch.float32, device=dev)
+        p_out = torch.empty_like(p_q)
+        p_maxq = int(wl.q_lens[pseq].max())
+        pairs = int((wl.positions[p_rows].astype(np.int64) + 1).sum())  # causal (query, key) pairs
+        prefill_flops = pairs * sp.Hq * sp.D * 4  # QK^T and PV, 2 flops per multiply-add
 
     def append():
         K.kv_append(pool, sp.layer, attn, q, k, v, tok_req, positions, bt, q_out, qn, kn, rope, wl.max_seq_len,
                     stream=stream)
 
+    def gather_q():
+        if B and B != T:
+            torch.index_select(q_out.view(T, sp.Hq, sp.D), 0, d_rows, out=d_q)
+        if prefill_flops:
+            torch.index_select(q_out.view(T, sp.Hq, sp.D), 0, p_rows_t, out=p_q)
+
+    def prefill():
+        if prefill_flops:
+            K.paged_prefill_attention(pool, sp.layer, attn, p_q, p_cu_t, p_ctx, p_bt, p_maxq, p_out, stream=stream)
+
     def decode():
-        K.paged_decode_attention(pool, sp.layer, attn, q_out.view(B, sp.Hq, sp.D), bt, ctx, mx, out, ws,
-                                 args.split_tokens, stream=stream)
+        if B:
+            K.paged_decode_attention(pool, sp.layer, attn, d_q, d_bt, d_ctx, mx, out, ws, args.split_tokens,
+                                     stream=stream)
 
     def barrier():
         if dist is not None:
             dist.barrier()
 
-    # ---- device-resident timing: K steps, events around every decode launch
-    for _ in range(max(args.warmup, 3)):
+    # ---- device-resident timing: K steps, events around every decode and prefill launch
+    def step(i=None):
         append()
+        gather_q()
+        if prefill_flops:
+            if i is not None:
+                evp[i][0].record(stream)
+            prefill()
+            if i is not None:
+                evp[i][1].record(stream)
+        if i is not None:
+            ev[i][0].record(stream)
         decode()
+        if i is not None:
+            ev[i][1].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
     pool.sync_status(stream)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    evp = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     clocks = ClockSampler(dev.index)
     clocks.start()
     barrier()
@@ -275,10 +329,7 @@ def run_ours(args):
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
     for i in range(args.steps):
-        append()
-        ev[i][0].record(stream)
-        decode()
-        ev[i][1].record(stream)
+        step(i)
     t_end.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -286,10 +337,8 @@ def run_ours(args):
     pool.sync_status(stream)
     step_ms = t_start.elapsed_time(t_end) / args.steps
     dec_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
-    if dist is not None:
-        t = torch.tensor([step_ms, dec_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_ms, dec_ms = float(t[0]), float(t[1])
+    pre_ms = float(np.mean([a.elapsed_time(b) for a, b in evp])) if prefill_flops else 0.0
+    step_ms, dec_ms, pre_ms = replicas.max_over_ranks([step_ms, dec_ms, pre_ms], dist, dev)
 
     # ---- end to end through the C ABI with host buffers: H2D of the step's
     # inputs from pinned memory, the step, D2H of the attention output
@@ -305,8 +354,7 @@ def run_ours(args):
     def e2e_step():
         for h, d in zip(h_in, d_in):
             d.copy_(h, non_blocking=True)
-        append()
-        decode()
+        step()
         h_out.copy_(out, non_blocking=True)
 
     for _ in range(3):
@@ -321,15 +369,12 @@ def run_ours(args):
     torch.cuda.synchronize()
     barrier()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if dist is not None:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t[0])
+    (e2e_ms,) = replicas.max_over_ranks([e2e_ms], dist, dev)
     pool.sync_status(stream)
 
     peak, peak_kind = measured_peaks()
     total_bytes = kv_bytes * world
-    value = total_bytes / (step_ms * 1e-3) / 1e9
+    value = replicas.job_throughput(kv_bytes, world, step_ms * 1e-3) / 1e9
     achieved = kv_bytes / (dec_ms * 1e-3) / 1e9
     traffic = ncu_traffic(args.workload)
     line = {
@@ -346,7 +391,7 @@ def run_ours(args):
         "dtype": sp.kv_dtype,
         "data": "synthetic",
         "config": {"workload": args.workload, "batch": B, "Hq": sp.Hq, "Hkv": sp.Hkv, "head_dim": sp.D,
-                   "block_size": sp.bs, "kv_dtype": sp.kv_dtype, "ctx_range": [int(wl.ctx.min()), mx],
+                   "block_size": sp.bs, "kv_dtype": sp.kv_dtype, "ctx_range": [int(wl.ctx[dseq].min()) if B else 0, mx],
                    "kv_bytes_per_step": kv_bytes, "split_tokens": args.split_tokens or "auto",
                    "l2": f"inputs larger than L2 ({kv_bytes / 1e6:.0f} MB of K/V per step vs 126 MB L2)",
                    "parallelism": f"replicas x{world}"},
@@ -362,9 +407,17 @@ def run_ours(args):
         "clocks": clk,
         "e2e": {"value": round(total_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": (2 + (1 if prefill_flops else 0)) * args.steps,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if prefill_flops:
+        bf16_peak = measured_bf16_tflops()
+        tf = prefill_flops / (pre_ms * 1e-3) / 1e12
+        line["prefill"] = {"kernel": "kvp::pre::prefill_kernel", "us": round(pre_ms * 1e3, 2),
+                           "flops_per_launch": prefill_flops, "tflops": round(tf, 2),
+                           "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": bf16_peak[0],
+                                        "unit": "TFLOP/s", "frac": round(tf / bf16_peak[0], 4),
+                                        "peak_kind": bf16_peak[1] + " bf16 (the fp16 dense rate is the same)"}}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not prefill_flops:
         line["cpu_baseline"] = cpu_baseline(wl)
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -1,0 +1,56 @@
+"""The C-ABI library loads without a GPU and exports every function that
+include/kvpaged.h declares (no compute calls: those need a GPU)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "kvpaged.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s*([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M)
+    return sorted(set(n for n in names if n not in ("if", "while")))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("kv_pool_create", "kv_append", "paged_decode_attention", "paged_prefill_attention"):
+        assert required in names
+    assert len(names) >= 15
+
+
+def test_library_exports_every_declared_symbol():
+    from paged_kv_cache_321_b200 import build
+
+    lib_path = build.build()
+    lib = ctypes.CDLL(lib_path)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    lib.kvp_version.restype = ctypes.c_int
+    assert lib.kvp_version() >= 100
+
+
+def test_binding_lists_every_export():
+    import paged_kv_cache_321_b200 as K
+
+    assert sorted(K.EXPORTS) == declared_functions()
+
+
+def test_host_side_errors_need_no_gpu():
+    # argument validation happens before any CUDA call
+    import paged_kv_cache_321_b200 as K
+
+    lib = K.lib()
+    out = ctypes.c_void_p()
+    rc = lib.kv_pool_create(None, None, None, ctypes.byref(out))
+    assert rc == K.KVP_EINVAL
+    assert b"NULL" in lib.kvp_last_error()
+    assert lib.kv_pool_destroy(None) == K.KVP_OK
+    cfg = K.AttnConfig(32, 8, 128, 5e5, 1e-6)
+    assert lib.kvp_rope_table_bytes(ctypes.byref(cfg), 100) == 100 * 128 * 4
+    assert lib.kvp_rope_table_fill(ctypes.byref(K.AttnConfig(32, 8, 127, 5e5, 1e-6)), 10, None) != 0
