@@ -24,7 +24,11 @@
  *     DEVICE pointer on the pool's device; the caller owns all memory (the
  *     library allocates only the pool handle and its 8-byte status word).
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
- *     default stream) unless stated otherwise.
+ *     default stream) unless stated otherwise. Kernels are launched with a
+ *     programmatic dependency on the stream's previous kernel: a grid may be
+ *     placed on the SMs while that kernel runs, but it touches no global
+ *     memory before that kernel has completed, so stream order holds exactly
+ *     as for plain launches.
  *   - Errors that the host can see (bad shapes, unsupported sizes, NULL
  *     pointers) are returned before anything is launched, with a message
  *     available from kvp_last_error().

@@ -30,9 +30,13 @@
 //    values at every step, leaving each lane with distinct (token, head)
 //    scores; one exp2 per score, P goes to the PV pass through shared memory;
 //  * a context split over several warps leaves (max, sum, unnormalised
-//    output) partials in the workspace; the warp that finishes the context
-//    last (atomic counter) combines them by log-sum-exp and resets the
-//    counter, so no second launch is needed.
+//    output) partials in the workspace and counts itself in with one
+//    acquire-release atomic; the warp that brings the count to the number
+//    of segments merges them by log-sum-exp and resets the counter, so no
+//    second launch (and no grid-wide drain before the merge) is needed. With
+//    8 query heads per kv head (no registers to spare) a second grid, one
+//    warp per (context, head), does the merge instead. A context inside one
+//    warp's range is normalised and written by that warp.
 #include <math.h>
 
 #include <type_traits>
@@ -85,8 +89,8 @@ struct Params {
     const int32_t *bt;        // [B][mbps]
     const int32_t *ctx;       // [B]
     float *out;               // [B][Hq][D]
-    float *part;              // [W + B*Hkv][G][D + 2]: output, then (max, sum) per head
-    int *counters;            // [B*Hkv]
+    float *part;              // [W + B*Hkv] slots of slot_floats(G, D): outputs, then (max, sum) per head
+    int *counters;            // [B*Hkv] segments finished per split context
     int *status;
     int B, Hq, Hkv, mbps, bs, num_blocks, max_ctx, max_seq_len, warps_total, min_tiles;
     float qscale;  // softmax scale * log2(e)
@@ -185,15 +189,152 @@ struct Cursor {
     int nt;  // tiles of sequence r
 };
 
-// Log-sum-exp combine of the partials of context (r, h), written by warps
-// w_first .. w_last into consecutive slots; one warp.
-template <int D, int G>
-__device__ void combine(const Params &p, int rhidx, int w_first, int w_last, int lane, float *out_rh)
+// A context length the kernels accept (else the row is zero and an error is
+// reported by the decode kernel).
+__device__ __forceinline__ bool ctx_ok(const Params &p, int c)
 {
-    constexpr int SL = G * (D + 2);
-    constexpr int DL = D / 32;  // dims per lane: 2, 4 or 8
+    return c >= 0 && c <= p.max_ctx && c <= p.mbps * p.bs && c <= p.max_seq_len;
+}
+
+// Exclusive prefix of s_tiles[i] * Hkv over the B sequences into s_pref[0..B],
+// by one warp; s_pref[B] is the length of the global tile sequence.
+__device__ __forceinline__ void tile_prefix(const int *s_tiles, int *s_pref, int B, int Hkv, int lane)
+{
+    int run = 0;
+    for (int base = 0; base < B; base += 32) {
+        const int i = base + lane;
+        const int v = i < B ? s_tiles[i] * Hkv : 0;
+        int x = v;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, off);
+            if (lane >= off) x += y;
+        }
+        if (i < B) s_pref[i] = run + x - v;
+        run += __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (lane == 0) s_pref[B] = run;
+}
+
+// Number of warps the global tile sequence of `total` tiles is cut over.
+__device__ __forceinline__ int active_warps(const Params &p, int total)
+{
+    return max(1, min(p.warps_total, (total + p.min_tiles - 1) / p.min_tiles));
+}
+
+// First and last warp whose range of the global tile sequence overlaps the
+// tiles [A, A + nt) of one context.
+__device__ __forceinline__ void context_warps(int A, int nt, int W, int total, int &w_first, int &w_last)
+{
+    w_first = static_cast<int>(((static_cast<int64_t>(A) + 1) * W - 1) / total);
+    w_last = static_cast<int>(((static_cast<int64_t>(A) + nt) * W - 1) / total);
+}
+
+// Floats in one partial-result slot: G output rows of D, then G (max, sum)
+// pairs padded to 16 bytes, so every slot and row starts 16-byte aligned.
+__host__ __device__ constexpr int slot_floats(int G, int D) { return G * D + ((2 * G + 3) & ~3); }
+
+// Partial-result slot of the segment of context rh computed by warp w: the
+// slots of one context's segments are consecutive (w_first + rh ...), and a
+// warp's two split segments (its first and its last) never collide with
+// another warp's, because contexts advance with the warp index.
+template <int D, int G>
+__device__ __forceinline__ float *part_slot(const Params &p, int w, int rh)
+{
+    return p.part + static_cast<size_t>(w + rh) * slot_floats(G, D);
+}
+
+// Log-sum-exp merge of the partials of context rh (query heads h*G ..
+// h*G+G-1), written by warps w_first .. w_last into consecutive slots; run by
+// one warp, the one that finished the context last, so its latency is the
+// tail of the kernel. One load round trip brings every segment's (max, sum)
+// pairs (lane = segment); the weights come from warp reductions; then the
+// (segment, head) output rows stream in chunks of CI rows per lane, each
+// chunk's loads all issued (predicated, no remainder loop) before the first
+// is used. Loads bypass L1: the partials were written on other SMs. Kept
+// out of line with a small chunk: its registers must not cost the streaming
+// loop any (a larger chunk made that loop spill).
+template <int D, int G>
+__device__ __noinline__ void combine(const Params &p, int rh, int w_first, int w_last, int lane, float *out_rh)
+{
+    constexpr int SL = slot_floats(G, D);
+    constexpr int DL = D / 32;                    // output dims per lane: 2, 4 or 8
+    constexpr int CI = cmax(G, 32 / DL);          // (segment, head) rows per chunk: 32 floats per lane
+    constexpr int CS = CI / G;                    // segments per chunk
+    using V = typename std::conditional<DL == 2, float2, float4>::type;
+    constexpr int NV = DL * 4 / static_cast<int>(sizeof(V));  // vectors per row and lane
     const int nseg = w_last - w_first + 1;
-    const float *base = p.part + static_cast<size_t>(w_first + rhidx) * SL;
+    const float *base = part_slot<D, G>(p, w_first, rh);
+    if (nseg <= 32) {
+        float m[G], l[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            m[g] = -INFINITY;
+            l[g] = 0.0f;
+        }
+        if (lane < nseg) {
+            const float2 *ml = reinterpret_cast<const float2 *>(base + static_cast<size_t>(lane) * SL + G * D);
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const float2 v = __ldcg(ml + g);
+                m[g] = v.x;
+                l[g] = v.y;
+            }
+        }
+        float w[G], L[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            float M = m[g];
+#pragma unroll
+            for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+            w[g] = (m[g] == -INFINITY) ? 0.0f : ex2(m[g] - M);
+            L[g] = l[g] * w[g];
+#pragma unroll
+            for (int off = 16; off; off >>= 1) L[g] += __shfl_xor_sync(0xffffffffu, L[g], off);
+        }
+        float acc[G][DL];
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int d = 0; d < DL; ++d) acc[g][d] = 0.0f;
+        const float *row0 = base + lane * DL;
+#pragma unroll 1
+        for (int s0 = 0; s0 < nseg; s0 += CS) {
+            V buf[CS][G][NV];
+#pragma unroll
+            for (int k = 0; k < CS; ++k) {
+                const bool live = s0 + k < nseg;
+                const float *srow = row0 + static_cast<size_t>(s0 + k) * SL;
+#pragma unroll
+                for (int g = 0; g < G; ++g)
+#pragma unroll
+                    for (int v = 0; v < NV; ++v) {
+                        if (live) buf[k][g][v] = __ldcg(reinterpret_cast<const V *>(srow + g * D) + v);
+                        else buf[k][g][v] = V{};
+                    }
+            }
+#pragma unroll
+            for (int k = 0; k < CS; ++k) {
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const float ws = __shfl_sync(0xffffffffu, w[g], min(s0 + k, 31));  // 0 past nseg
+                    const float *f = reinterpret_cast<const float *>(buf[k][g]);
+#pragma unroll
+                    for (int d = 0; d < DL; ++d) acc[g][d] = fmaf(f[d], ws, acc[g][d]);
+                }
+            }
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float inv = L[g] > 0.0f ? 1.0f / L[g] : 0.0f;
+#pragma unroll
+            for (int d = 0; d < DL; d += 2)
+                *reinterpret_cast<float2 *>(out_rh + g * D + lane * DL + d) =
+                    make_float2(acc[g][d] * inv, acc[g][d + 1] * inv);
+        }
+        return;
+    }
+    // more than 32 segments: per head, max, sum, then the outputs
 #pragma unroll 1
     for (int g = 0; g < G; ++g) {
         float M = -INFINITY;
@@ -202,9 +343,8 @@ __device__ void combine(const Params &p, int rhidx, int w_first, int w_last, int
         for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
         float L = 0.0f;
         for (int s = lane; s < nseg; s += 32) {
-            const float *ml = base + static_cast<size_t>(s) * SL + G * D + 2 * g;
-            const float m = __ldcg(ml);
-            L += (m == -INFINITY) ? 0.0f : __ldcg(ml + 1) * ex2(m - M);
+            const float2 v = __ldcg(reinterpret_cast<const float2 *>(base + static_cast<size_t>(s) * SL + G * D) + g);
+            L += (v.x == -INFINITY) ? 0.0f : v.y * ex2(v.x - M);
         }
 #pragma unroll
         for (int off = 16; off; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
@@ -212,7 +352,7 @@ __device__ void combine(const Params &p, int rhidx, int w_first, int w_last, int
         float acc[DL];
 #pragma unroll
         for (int d = 0; d < DL; ++d) acc[d] = 0.0f;
-#pragma unroll 4
+#pragma unroll 8
         for (int s = 0; s < nseg; ++s) {
             const float *sl = base + static_cast<size_t>(s) * SL;
             const float m = __ldcg(sl + G * D + 2 * g);
@@ -229,6 +369,27 @@ __device__ void combine(const Params &p, int rhidx, int w_first, int w_last, int
         for (int d = 0; d < DL; d += 2)
             *reinterpret_cast<float2 *>(out_rh + g * D + lane * DL + d) = make_float2(acc[d] * inv, acc[d + 1] * inv);
     }
+}
+
+// With 8 query heads per kv head the streaming loop already needs every
+// register a thread can have; any merge code inside it costs spills there.
+// Those contexts are merged by a separate grid instead (combine_kernel),
+// one warp per (context, head), so a context's merge is also spread over
+// G warps rather than run by one.
+template <int G>
+struct GridCombine {
+    static constexpr bool value = G >= 8;
+};
+
+// Atomic add at GPU scope with acquire-release semantics: the release makes
+// this warp's partial (ordered before it by __syncwarp) visible before the
+// count moves; the acquire makes every earlier contributor's partial
+// visible to the warp that sees the final count.
+__device__ __forceinline__ int atomic_add_acq_rel(int *addr, int v)
+{
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v) : "memory");
+    return old;
 }
 
 template <int D, int G, bool BF16>
@@ -250,10 +411,14 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int B = p.B, Hkv = p.Hkv;
 
+    // Nothing global is touched before the previous grid on the stream has
+    // completed: with a programmatic launch only the launch itself overlaps.
+    grid_dependency_wait();
+
     // ---- tiles per sequence; invalid or empty sequences get none and a zero row
     for (int i = tid; i < B; i += NW * 32) {
         const int c = p.ctx[i];
-        const bool ok = c >= 0 && c <= p.max_ctx && c <= p.mbps * p.bs && c <= p.max_seq_len;
+        const bool ok = ctx_ok(p, c);
         s_tiles[i] = ok ? (c + TT - 1) / TT : 0;
         if (blockIdx.x == 0 && (!ok || c == 0)) {
             if (!ok) report(p.status, KVP_ERANGE, i);
@@ -262,28 +427,14 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
         }
     }
     __syncthreads();
-    // ---- exclusive prefix of tiles * Hkv over the sequences (warp 0)
-    if (warp == 0) {
-        int run = 0;
-        for (int base = 0; base < B; base += 32) {
-            const int i = base + lane;
-            const int v = i < B ? s_tiles[i] * Hkv : 0;
-            int x = v;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, x, off);
-                if (lane >= off) x += y;
-            }
-            if (i < B) s_pref[i] = run + x - v;
-            run += __shfl_sync(0xffffffffu, x, 31);
-        }
-        if (lane == 0) s_pref[B] = run;
-    }
+    if (warp == 0) tile_prefix(s_tiles, s_pref, B, Hkv, lane);
     __syncthreads();
+
+    grid_launch_dependents();  // the next grid may be placed (it waits for this one)
 
     // ---- this warp's share of the global tile sequence
     const int total = s_pref[B];
-    const int W = max(1, min(p.warps_total, (total + p.min_tiles - 1) / p.min_tiles));
+    const int W = active_warps(p, total);
     const int w = blockIdx.x * NW + warp;
     if (w >= W) return;
     const int t_begin = static_cast<int>(static_cast<int64_t>(w) * total / W);
@@ -651,12 +802,11 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
             const int obase = halving_base<S::NO, S::OLEV>(lane, LPT);
             // the warps covering this context's global tiles [A, A + nt)
             const int A = s_pref[r] + h * nt;
-            const int w_first = static_cast<int>(((static_cast<int64_t>(A) + 1) * W - 1) / total);
-            const int w_last = static_cast<int>(((static_cast<int64_t>(A) + nt) * W - 1) / total);
+            int w_first, w_last;
+            context_warps(A, nt, W, total, w_first, w_last);
             float *out_rh = p.out + (static_cast<size_t>(r) * p.Hq + static_cast<size_t>(h) * G) * D;
             const bool whole = (w_first == w_last);
-            const int rhidx = r * Hkv + h;
-            float *slot = p.part + static_cast<size_t>(w + rhidx) * G * (D + 2);
+            float *slot = part_slot<D, G>(p, w, r * Hkv + h);
 #pragma unroll
             for (int x = 0; x < S::OVPL; ++x) {
                 const int k = obase + x;
@@ -681,19 +831,132 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
                     slot[G * D + lane * 2 + 0] = mg;
                     slot[G * D + lane * 2 + 1] = lg;
                 }
-                __threadfence();
-                __syncwarp();
-                int last = 0;
-                if (lane == 0) last = atomicAdd(&p.counters[rhidx], 1) == (w_last - w_first);
-                last = __shfl_sync(0xffffffffu, last, 0);
-                if (last) {
-                    __threadfence();
-                    combine<D, G>(p, rhidx, w_first, w_last, lane, out_rh);
-                    if (lane == 0) p.counters[rhidx] = 0;
+                if constexpr (!GridCombine<G>::value) {
+                    __syncwarp();
+                    const int rh = r * Hkv + h;
+                    int last = 0;
+                    if (lane == 0) last = atomic_add_acq_rel(&p.counters[rh], 1) == (w_last - w_first);
+                    last = __shfl_sync(0xffffffffu, last, 0);
+                    if (last) {
+                        __syncwarp();  // lane 0's acquire orders the other lanes' loads too
+                        combine<D, G>(p, rh, w_first, w_last, lane, out_rh);
+                        if (lane == 0) p.counters[rh] = 0;  // ready for the next call
+                    }
                 }
             }
         }
         advance(cons);
+    }
+}
+
+
+
+// ------------------------------------------------------------ combine grid
+// Log-sum-exp merge for GridCombine group sizes: one warp per (context,
+// query head of the group). All segments' (max, sum) pairs come in one load
+// (lane = segment), then all segments' output rows in one batch of loads.
+// Launched right after the decode grid with a programmatic dependency, so
+// its launch and the prefix over the context lengths overlap the decode
+// grid's tail.
+constexpr int kCombineWarps = 8;
+
+template <int D, int G>
+__global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const Params p)
+{
+    constexpr int SL = slot_floats(G, D);
+    constexpr int DL = D / 32;  // output dims per lane: 2, 4 or 8
+    extern __shared__ __align__(16) int csm[];
+    int *s_tiles = csm;
+    int *s_pref = csm + p.B;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int B = p.B, Hkv = p.Hkv;
+
+    // The context lengths were final before the decode grid started (it
+    // waited for its predecessor), so they may be read before it finishes.
+    for (int i = tid; i < B; i += kCombineWarps * 32) {
+        const int c = p.ctx[i];
+        s_tiles[i] = ctx_ok(p, c) ? (c + TT - 1) / TT : 0;
+    }
+    __syncthreads();
+    if (warp == 0) tile_prefix(s_tiles, s_pref, B, Hkv, lane);
+    __syncthreads();
+    const int total = s_pref[B];
+    const int W = active_warps(p, total);
+
+    grid_dependency_wait();  // the partials are complete and visible
+    grid_launch_dependents();
+
+    const int ntask = B * Hkv * G;
+    for (int task = blockIdx.x * kCombineWarps + warp; task < ntask; task += gridDim.x * kCombineWarps) {
+        const int g = task % G, rh = task / G;
+        const int r = rh / Hkv, h = rh - r * Hkv;
+        const int nt = s_tiles[r];
+        if (nt == 0) continue;
+        int w_first, w_last;
+        context_warps(s_pref[r] + h * nt, nt, W, total, w_first, w_last);
+        if (w_first == w_last) continue;  // written by the decode grid itself
+        const int nseg = w_last - w_first + 1;
+        const float *base = part_slot<D, G>(p, w_first, rh);
+
+        // (max, sum) of the segments; lane s keeps segment s
+        float m0 = -INFINITY, l0 = 0.0f;
+        if (lane < nseg) {
+            const float2 v = __ldcg(reinterpret_cast<const float2 *>(base + static_cast<size_t>(lane) * SL + G * D) + g);
+            m0 = v.x;
+            l0 = v.y;
+        }
+        float M = m0;
+        for (int s = lane + 32; s < nseg; s += 32) M = fmaxf(M, __ldcg(base + static_cast<size_t>(s) * SL + G * D + 2 * g));
+#pragma unroll
+        for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+        const float w0 = (m0 == -INFINITY) ? 0.0f : ex2(m0 - M);
+        float L = l0 * w0;
+        for (int s = lane + 32; s < nseg; s += 32) {
+            const float2 v = __ldcg(reinterpret_cast<const float2 *>(base + static_cast<size_t>(s) * SL + G * D) + g);
+            L += (v.x == -INFINITY) ? 0.0f : v.y * ex2(v.x - M);
+        }
+#pragma unroll
+        for (int off = 16; off; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+
+        // weighted sum of the segments' rows of head g; lane owns DL dims
+        float acc[DL];
+#pragma unroll
+        for (int d = 0; d < DL; ++d) acc[d] = 0.0f;
+        const float *row = base + g * D + lane * DL;
+        constexpr int CS = 8;  // segments per batch of loads
+#pragma unroll 1
+        for (int s0 = 0; s0 < nseg; s0 += CS) {
+            float buf[CS][DL];
+#pragma unroll
+            for (int k = 0; k < CS; ++k) {
+                const float *src = row + static_cast<size_t>(s0 + k) * SL;
+#pragma unroll
+                for (int d = 0; d < DL; d += 2) {
+                    float2 v = make_float2(0.0f, 0.0f);
+                    if (s0 + k < nseg) v = __ldcg(reinterpret_cast<const float2 *>(src + d));
+                    buf[k][d] = v.x;
+                    buf[k][d + 1] = v.y;
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < CS; ++k) {
+                const int s = s0 + k;
+                float ws;
+                if (s < 32) {
+                    ws = __shfl_sync(0xffffffffu, w0, s & 31);  // 0 past nseg
+                } else {
+                    const float m = s < nseg ? __ldcg(base + static_cast<size_t>(s) * SL + G * D + 2 * g) : -INFINITY;
+                    ws = (m == -INFINITY) ? 0.0f : ex2(m - M);
+                }
+#pragma unroll
+                for (int d = 0; d < DL; ++d) acc[d] = fmaf(buf[k][d], ws, acc[d]);
+            }
+        }
+        const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+        float *dst = p.out + (static_cast<size_t>(r) * p.Hq + static_cast<size_t>(h) * G + g) * D + lane * DL;
+#pragma unroll
+        for (int d = 0; d < DL; d += 2)
+            *reinterpret_cast<float2 *>(dst + d) = make_float2(acc[d] * inv, acc[d + 1] * inv);
     }
 }
 
@@ -742,7 +1005,7 @@ static int plan(const kvp_pool *pool, int G, int Hkv, int B, int max_ctx, int sp
     L->warps_total = sms * nw;
     L->min_tiles = split_req > 0 ? split_req / TT : kAutoMinTiles;
     const size_t rh = static_cast<size_t>(B) * Hkv;
-    const size_t slot = static_cast<size_t>(G) * (pool->cfg.head_dim + 2) * 4;
+    const size_t slot = static_cast<size_t>(slot_floats(G, pool->cfg.head_dim)) * 4;
     L->counters = 0;
     L->part = align_up(rh * 4, 256);
     L->total = align_up(L->part + (L->warps_total + rh) * slot, 256);
@@ -758,8 +1021,16 @@ static int launch(const Params &p, bool bf16, int blocks, cudaStream_t s)
     int rc = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)),
                         "decode smem attribute");
     if (rc) return rc;
-    kern<<<blocks, Shape<D, G>::NW * 32, smem, s>>>(p);
-    return check_cuda(cudaGetLastError(), "decode launch");
+    if ((rc = check_cuda(launch_pdl(kern, dim3(blocks), dim3(Shape<D, G>::NW * 32), smem, s, p), "decode launch")))
+        return rc;
+    if constexpr (GridCombine<G>::value) {
+        const int tasks = p.B * p.Hkv * G;
+        const int cblocks = max(1, min((tasks + kCombineWarps - 1) / kCombineWarps, 4 * blocks));
+        const size_t csmem = align_up(sizeof(int) * (2 * static_cast<size_t>(p.B) + 1), 16);
+        rc = check_cuda(launch_pdl(combine_kernel<D, G>, dim3(cblocks), dim3(kCombineWarps * 32), csmem, s, p),
+                        "decode combine launch");
+    }
+    return rc;
 }
 
 template <int D>

@@ -84,6 +84,10 @@ __global__ void __launch_bounds__(kAppendWarps * 32) kv_append_kernel(const Appe
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
     const int R = p.Hq + 2 * p.Hkv;
     const int64_t row = static_cast<int64_t>(blockIdx.x) * kAppendWarps + wib;
+    // launched with a programmatic dependency: wait for the previous grid's
+    // results, then let the next grid launch (it waits for this one in turn)
+    grid_dependency_wait();
+    grid_launch_dependents();
     if (row >= static_cast<int64_t>(p.T) * R) return;
     const int t = static_cast<int>(row / R), rr = static_cast<int>(row % R);
     const int kind = rr < p.Hq ? 0 : (rr < p.Hq + p.Hkv ? 1 : 2);  // q, k, v
@@ -164,14 +168,12 @@ __global__ void __launch_bounds__(kAppendWarps * 32) kv_append_kernel(const Appe
 }
 
 template <int D>
-static void launch_append(const AppendParams &p, bool bf16, cudaStream_t s)
+static cudaError_t launch_append(const AppendParams &p, bool bf16, cudaStream_t s)
 {
     const int64_t rows = static_cast<int64_t>(p.T) * (p.Hq + 2 * p.Hkv);
     const unsigned blocks = static_cast<unsigned>((rows + kAppendWarps - 1) / kAppendWarps);
-    if (bf16)
-        kv_append_kernel<D, true><<<blocks, kAppendWarps * 32, 0, s>>>(p);
-    else
-        kv_append_kernel<D, false><<<blocks, kAppendWarps * 32, 0, s>>>(p);
+    return launch_pdl(bf16 ? kv_append_kernel<D, true> : kv_append_kernel<D, false>, dim3(blocks),
+                      dim3(kAppendWarps * 32), 0, s, p);
 }
 
 }  // namespace kvp
@@ -214,10 +216,9 @@ extern "C" int kv_append(kvp_pool *pool, int layer, const kvp_attn_config *attn,
     const bool bf16 = pool->cfg.kv_dtype == KVP_BF16;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     switch (D) {
-    case 64: launch_append<64>(p, bf16, s); break;
-    case 128: launch_append<128>(p, bf16, s); break;
-    case 256: launch_append<256>(p, bf16, s); break;
+    case 64: return check_cuda(launch_append<64>(p, bf16, s), "kv_append launch");
+    case 128: return check_cuda(launch_append<128>(p, bf16, s), "kv_append launch");
+    case 256: return check_cuda(launch_append<256>(p, bf16, s), "kv_append launch");
     default: return set_error(KVP_EUNSUPPORTED, "head_dim %d", D);
     }
-    return check_cuda(cudaGetLastError(), "kv_append launch");
 }

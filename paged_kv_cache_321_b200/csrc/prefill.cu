@@ -210,6 +210,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(smem + TMEM_PTR_OFF);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // launched with a programmatic dependency: nothing global is read before
+    // the previous grid has completed
+    grid_dependency_wait();
+    grid_launch_dependents();
     // blockIdx: x = query tile (largest first), y = kv head, z = sequence
     const int s = blockIdx.z, h = blockIdx.y, qt = p.ntq - 1 - blockIdx.x;
     const int q0 = p.cu_q[s], q_len = p.cu_q[s + 1] - q0;
@@ -516,9 +520,8 @@ static int launch(const CUtensorMap &mk, const CUtensorMap &mv, const Params &p,
     int rc = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES),
                         "prefill smem attribute");
     if (rc) return rc;
-    dim3 grid(p.ntq, p.Hkv, p.S);
-    kern<<<grid, NTHREADS, SMEM_BYTES, s>>>(mk, mv, p);
-    return check_cuda(cudaGetLastError(), "prefill launch");
+    return check_cuda(launch_pdl(kern, dim3(p.ntq, p.Hkv, p.S), dim3(NTHREADS), SMEM_BYTES, s, mk, mv, p),
+                      "prefill launch");
 }
 
 }  // namespace pre

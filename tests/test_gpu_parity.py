@@ -123,6 +123,32 @@ def test_split_invariance_and_single_split_identity(orc, dev):
         assert_close(out.cpu().numpy(), one.cpu().numpy(), f"split {split} vs 1")
 
 
+@pytest.mark.parametrize("name", ["gqa8-long", "llama-ragged"])
+def test_workspace_reuse_is_bitwise_stable(orc, dev, name):
+    # a zero-filled workspace reused by calls of different split sizes and
+    # batch sizes gives the same bits as a fresh one each time: every call
+    # leaves its split counters (the first B*Hkv int32 words) at zero
+    import paged_kv_cache_321_b200 as K
+    wl = make_workload(SMALL[name])
+    run = GpuRun(wl, dev)
+    run.append()
+    q, bt, ctx, mx = run.decode_inputs()
+    B, Hkv = ctx.numel(), wl.spec.Hkv
+    n = max(K.decode_workspace_size(run.pool, run.attn, B, mx, sp) for sp in (16, 0))
+    shared = torch.zeros(n // 4 + 64, dtype=torch.float32, device=dev)
+    one = (q[:1].contiguous(), bt[:1].contiguous(), ctx[:1].contiguous(), int(wl.ctx[wl.decode_seqs[0]]))
+    calls = [((q, bt, ctx, mx), 16), ((q, bt, ctx, mx), 16), ((q, bt, ctx, mx), 0), (one, 16), ((q, bt, ctx, mx), 16)]
+    for args, split in calls:
+        out = torch.empty_like(args[0])
+        K.paged_decode_attention(run.pool, 0, run.attn, *args, out, shared, split)
+        fresh = torch.zeros_like(shared)
+        ref = torch.empty_like(args[0])
+        K.paged_decode_attention(run.pool, 0, run.attn, *args, ref, fresh, split)
+        run.pool.sync_status()
+        assert np.array_equal(out.cpu().numpy().view(np.uint32), ref.cpu().numpy().view(np.uint32)), split
+        assert not shared.view(torch.int32)[:B * Hkv].any().item(), "split counters not reset"
+
+
 def test_decode_special_cases(orc, dev):
     wl = make_workload(SMALL["llama-ragged"])
     run = GpuRun(wl, dev)
