@@ -30,13 +30,16 @@
 //    values at every step, leaving each lane with distinct (token, head)
 //    scores; one exp2 per score, P goes to the PV pass through shared memory;
 //  * a context split over several warps leaves (max, sum, unnormalised
-//    output) partials in the workspace and counts itself in with one
-//    acquire-release atomic; the warp that brings the count to the number
-//    of segments merges them by log-sum-exp and resets the counter, so no
-//    second launch (and no grid-wide drain before the merge) is needed. With
-//    8 query heads per kv head (no registers to spare) a second grid, one
-//    warp per (context, head), does the merge instead. A context inside one
-//    warp's range is normalised and written by that warp.
+//    output) partials in the workspace and counts them in after a release
+//    fence (the count's reply is looked at only at the end of the range, so
+//    the stream does not wait for it); the warp that brings a count to the
+//    number of segments merges them by log-sum-exp and resets the counter,
+//    so no second launch (and no grid-wide drain before the merge) is
+//    needed. With 8 query heads per kv head (no registers to spare) a second
+//    grid, one warp per (context, head), does the merge instead. A context
+//    inside one warp's range is normalised and written by that warp;
+//  * the first tile of each segment also brings the segment's queries into
+//    L1 (prefetch), and the K/V copies carry an L2 evict-first policy.
 #include <math.h>
 
 #include <type_traits>
@@ -381,14 +384,16 @@ struct GridCombine {
     static constexpr bool value = G >= 8;
 };
 
-// Atomic add at GPU scope with acquire-release semantics: the release makes
-// this warp's partial (ordered before it by __syncwarp) visible before the
-// count moves; the acquire makes every earlier contributor's partial
-// visible to the warp that sees the final count.
-__device__ __forceinline__ int atomic_add_acq_rel(int *addr, int v)
+// GPU-scope fence with acquire-release semantics. Before a count: this
+// warp's partials (ordered before it by __syncwarp) are visible before the
+// count moves. After the final count: every earlier contributor's partial is
+// visible to the warp that merges.
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
+__device__ __forceinline__ int atomic_add_relaxed(int *addr, int v)
 {
     int old;
-    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v) : "memory");
+    asm volatile("atom.relaxed.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v) : "memory");
     return old;
 }
 
@@ -414,6 +419,15 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
     // Nothing global is touched before the previous grid on the stream has
     // completed: with a programmatic launch only the launch itself overlaps.
     grid_dependency_wait();
+
+    // ---- start the block table on its way to L2 (this CTA's share of it)
+    // while the context lengths are read; the copy descriptors read it next
+    {
+        const int64_t lines = (static_cast<int64_t>(B) * p.mbps * 4 + 127) / 128;
+        const int64_t lo = lines * blockIdx.x / gridDim.x, hi = lines * (blockIdx.x + 1) / gridDim.x;
+        const char *bt_bytes = reinterpret_cast<const char *>(p.bt);
+        for (int64_t l = lo + tid; l < hi && l < lo + 4 * NW * 32; l += NW * 32) prefetch_l2(bt_bytes + l * 128);
+    }
 
     // ---- tiles per sequence; invalid or empty sequences get none and a zero row
     for (int i = tid; i < B; i += NW * 32) {
@@ -481,20 +495,24 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
     const size_t blk_stride = static_cast<size_t>(Hkv) * p.bs * D;
     const bool big_blocks = p.bs >= TT;  // a tile lies inside one block
     const int ntile = t_end - t_begin;
+    const uint64_t l2pol = l2_evict_first_policy();
 
     // Copy descriptors of 32 consecutive tiles, one per lane: the element
     // offset of the tile's K (and V) run in the layer pool and its number of
     // valid tokens (0: block id outside the pool).
     int64_t d_off = 0;
-    int d_nv = 0, dbase = 0;
+    int d_nv = 0, dbase = 0, d_q = -1;
     auto load_desc = [&](int base) {
         dbase = base;
         d_off = 0;
         d_nv = 0;
+        d_q = -1;
         const int i = base + lane;
         if (big_blocks && i < ntile) {
             Cursor c;
             locate(t_begin + i, c);
+            // a segment starts here: its queries are wanted when this tile is
+            if (c.ti == 0 || i == 0) d_q = c.r * p.Hq + c.h * G;
             const int ctx = p.ctx[c.r];
             const int tb = c.ti * TT;
             const int blk = p.bt[static_cast<size_t>(c.r) * p.mbps + tb / p.bs];
@@ -533,8 +551,8 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
             mbar_arrive_expect_tx(bar, bytes);
             for (int t = 0; t < nv; t += p.bs) {
                 const int b = btr[(tb + t) / p.bs];
-                bulk_g2s(smem_addr(dst + t * D), src + b * blk_stride + static_cast<size_t>(c.h) * p.bs * D,
-                         p.bs * D * 2, bar);
+                bulk_g2s_hint(smem_addr(dst + t * D), src + b * blk_stride + static_cast<size_t>(c.h) * p.bs * D,
+                              p.bs * D * 2, bar, l2pol);
             }
         } else {
             mbar_arrive(bar);
@@ -547,13 +565,20 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
             if (i - dbase >= 32) load_desc(i);
             const int64_t off = __shfl_sync(0xffffffffu, d_off, i - dbase);
             const int nv = __shfl_sync(0xffffffffu, d_nv, i - dbase);
+            if (half == 0) {
+                // the first tile of a segment: bring its G query rows into L1
+                // now, so the segment does not start with an L2 round trip
+                const int qrow = __shfl_sync(0xffffffffu, d_q, i - dbase);
+                if (qrow >= 0)
+                    for (int l = lane; l < G * D / 32; l += 32) prefetch_l1(p.q + static_cast<size_t>(qrow) * D + l * 32);
+            }
             if (lane == 0) {
                 fence_proxy_async_smem();
                 const uint32_t bar = kbar0 + (st * 2 + half) * 8;
                 if (nv > 0) {
                     mbar_arrive_expect_tx(bar, S::TILE_WORDS * 2);
-                    bulk_g2s(smem_addr(wst + st * (S::STAGE_BYTES / 2) + half * S::TILE_WORDS),
-                             (half ? p.vp : p.kp) + off, S::TILE_WORDS * 2, bar);
+                    bulk_g2s_hint(smem_addr(wst + st * (S::STAGE_BYTES / 2) + half * S::TILE_WORDS),
+                                  (half ? p.vp : p.kp) + off, S::TILE_WORDS * 2, bar, l2pol);
                 } else {
                     mbar_arrive(bar);
                 }
@@ -589,6 +614,12 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
     float2 q2[G][4];
     float2 o2[G][4];
     float m_run[G], l_run[G];
+    // Split segments to count in: (context, first warp, last warp) of the
+    // range's first (0) and last (1) one. The first is counted in when it
+    // ends, but the count's old value (lane 0) is looked at only at the end
+    // of the range, so the stream does not wait for the atomic's reply; the
+    // last is counted in at the end of the range.
+    int npub = 0, rh0 = 0, wf0 = 0, wl0 = 0, rh1 = 0, wf1 = 0, wl1 = 0, old0 = -1;
 
     for (int seq = 0; seq < ntile; ++seq) {
         if (seq == 0 || cons.ti == 0) {  // a new context segment starts
@@ -832,20 +863,54 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
                     slot[G * D + lane * 2 + 1] = lg;
                 }
                 if constexpr (!GridCombine<G>::value) {
-                    __syncwarp();
-                    const int rh = r * Hkv + h;
-                    int last = 0;
-                    if (lane == 0) last = atomic_add_acq_rel(&p.counters[rh], 1) == (w_last - w_first);
-                    last = __shfl_sync(0xffffffffu, last, 0);
-                    if (last) {
-                        __syncwarp();  // lane 0's acquire orders the other lanes' loads too
-                        combine<D, G>(p, rh, w_first, w_last, lane, out_rh);
-                        if (lane == 0) p.counters[rh] = 0;  // ready for the next call
+                    // counted in at the end of the range (below), together
+                    // with the range's other split segment, so the stream
+                    // never waits on the count here
+                    if (npub++ == 0) {
+                        rh0 = r * Hkv + h, wf0 = w_first, wl0 = w_last;
+                        if (seq != ntile - 1) {
+                            __syncwarp();
+                            if (lane == 0) {
+                                fence_acq_rel_gpu();
+                                old0 = atomic_add_relaxed(&p.counters[rh0], 1);
+                            }
+                        }
+                    } else {
+                        rh1 = r * Hkv + h, wf1 = w_first, wl1 = w_last;
                     }
                 }
             }
         }
         advance(cons);
+    }
+
+    if constexpr (!GridCombine<G>::value) {
+        // Publish this warp's split segments (at most two: the range's first
+        // and last): one release fence for all partials written above, then
+        // the counts. The warp that completes a context merges it.
+        if (npub > 0) {
+            __syncwarp();
+            int last0 = 0, last1 = 0;
+            if (lane == 0) {
+                fence_acq_rel_gpu();
+                if (old0 < 0) old0 = atomic_add_relaxed(&p.counters[rh0], 1);  // not counted in yet
+                const int old1 = npub > 1 ? atomic_add_relaxed(&p.counters[rh1], 1) : -1;
+                last0 = old0 == wl0 - wf0;
+                last1 = npub > 1 && old1 == wl1 - wf1;
+                if (last0 || last1) fence_acq_rel_gpu();  // the other contributors' partials
+            }
+            last0 = __shfl_sync(0xffffffffu, last0, 0);
+            last1 = __shfl_sync(0xffffffffu, last1, 0);
+            __syncwarp();  // lane 0's acquire orders the other lanes' loads too
+            if (last0) {
+                combine<D, G>(p, rh0, wf0, wl0, lane, p.out + static_cast<size_t>(rh0) * G * D);
+                if (lane == 0) p.counters[rh0] = 0;  // ready for the next call
+            }
+            if (last1) {
+                combine<D, G>(p, rh1, wf1, wl1, lane, p.out + static_cast<size_t>(rh1) * G * D);
+                if (lane == 0) p.counters[rh1] = 0;
+            }
+        }
     }
 }
 
