@@ -110,7 +110,8 @@ struct Smem {
     static constexpr size_t pbuf = align_up(masks + S::NW * NST * 4, 16);
     static constexpr size_t tiles = pbuf + S::NW * TT * G * 8;  // [B] tiles per sequence
     __host__ __device__ static size_t pref(int B) { return align_up(tiles + 4 * static_cast<size_t>(B), 16); }  // [B + 1]
-    __host__ __device__ static size_t total(int B) { return align_up(pref(B) + 4 * static_cast<size_t>(B + 1), 128); }
+    __host__ __device__ static size_t cpref(int B) { return align_up(pref(B) + 4 * static_cast<size_t>(B + 1), 16); }  // [B + 1]
+    __host__ __device__ static size_t total(int B) { return align_up(cpref(B) + 4 * static_cast<size_t>(B + 1), 128); }
 };
 
 __device__ __forceinline__ float ex2(float x)
@@ -199,24 +200,36 @@ __device__ __forceinline__ bool ctx_ok(const Params &p, int c)
     return c >= 0 && c <= p.max_ctx && c <= p.mbps * p.bs && c <= p.max_seq_len;
 }
 
-// Exclusive prefix of s_tiles[i] * Hkv over the B sequences into s_pref[0..B],
-// by one warp; s_pref[B] is the length of the global tile sequence.
-__device__ __forceinline__ void tile_prefix(const int *s_tiles, int *s_pref, int B, int Hkv, int lane)
+// Cost of starting a context on a warp, in tiles: a warp whose range crosses
+// a context boundary pays for a second segment end (reductions, partial
+// write, fence) and a cold first tile, about one tile's time. The warps'
+// ranges are cut evenly in cost space, where every context is preceded by
+// kCtxCost empty units, so such a warp gets about one tile less.
+constexpr int kCtxCost = 1;
+
+// Exclusive prefixes over the B sequences, by one warp: s_pref[i] of the
+// tiles (s_tiles * Hkv), s_cpref[i] of the cost units (Hkv * (tiles +
+// kCtxCost) for a sequence with tiles). s_pref[B] is the number of tiles,
+// s_cpref[B] the length of the cost space.
+__device__ __forceinline__ void tile_prefix(const int *s_tiles, int *s_pref, int *s_cpref, int B, int Hkv, int lane)
 {
-    int run = 0;
+    int run = 0, crun = 0;
     for (int base = 0; base < B; base += 32) {
         const int i = base + lane;
-        const int v = i < B ? s_tiles[i] * Hkv : 0;
-        int x = v;
+        const int nt = i < B ? s_tiles[i] : 0;
+        const int v = nt * Hkv, cv = nt > 0 ? (nt + kCtxCost) * Hkv : 0;
+        int x = v, cx = cv;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
             const int y = __shfl_up_sync(0xffffffffu, x, off);
-            if (lane >= off) x += y;
+            const int cy = __shfl_up_sync(0xffffffffu, cx, off);
+            if (lane >= off) x += y, cx += cy;
         }
-        if (i < B) s_pref[i] = run + x - v;
+        if (i < B) s_pref[i] = run + x - v, s_cpref[i] = crun + cx - cv;
         run += __shfl_sync(0xffffffffu, x, 31);
+        crun += __shfl_sync(0xffffffffu, cx, 31);
     }
-    if (lane == 0) s_pref[B] = run;
+    if (lane == 0) s_pref[B] = run, s_cpref[B] = crun;
 }
 
 // Number of warps the global tile sequence of `total` tiles is cut over.
@@ -225,12 +238,31 @@ __device__ __forceinline__ int active_warps(const Params &p, int total)
     return max(1, min(p.warps_total, (total + p.min_tiles - 1) / p.min_tiles));
 }
 
-// First and last warp whose range of the global tile sequence overlaps the
-// tiles [A, A + nt) of one context.
-__device__ __forceinline__ void context_warps(int A, int nt, int W, int total, int &w_first, int &w_last)
+// Warp w owns the cost units [floor(w*TC/W), floor((w+1)*TC/W)). The first
+// tile whose cost position is at least U (the tiles of context (r, h) sit at
+// cost positions s_cpref[r] + h*(nt + kCtxCost) + kCtxCost + i).
+__device__ __forceinline__ int cost_to_tile(int64_t U, const int *s_tiles, const int *s_pref, const int *s_cpref,
+                                            int B)
 {
-    w_first = static_cast<int>(((static_cast<int64_t>(A) + 1) * W - 1) / total);
-    w_last = static_cast<int>(((static_cast<int64_t>(A) + nt) * W - 1) / total);
+    if (U >= s_cpref[B]) return s_pref[B];
+    int lo = 0, hi = B;  // s_cpref[lo] <= U < s_cpref[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s_cpref[mid] <= U) lo = mid;
+        else hi = mid;
+    }
+    const int nt = s_tiles[lo], span = nt + kCtxCost;
+    const int local = static_cast<int>(U - s_cpref[lo]);
+    const int h = local / span, off = local - h * span;
+    return s_pref[lo] + h * nt + max(0, off - kCtxCost);
+}
+
+// First and last warp whose cost range holds a tile of the context whose
+// first tile sits at cost position P (nt tiles); TC is the cost-space length.
+__device__ __forceinline__ void context_warps(int P, int nt, int W, int TC, int &w_first, int &w_last)
+{
+    w_first = static_cast<int>(((static_cast<int64_t>(P) + 1) * W - 1) / TC);
+    w_last = static_cast<int>(((static_cast<int64_t>(P) + nt) * W - 1) / TC);
 }
 
 // Floats in one partial-result slot: G output rows of D, then G (max, sum)
@@ -412,6 +444,7 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
     float2 *pbuf = reinterpret_cast<float2 *>(smem + M::pbuf);
     int *s_tiles = reinterpret_cast<int *>(smem + M::tiles);
     int *s_pref = reinterpret_cast<int *>(smem + M::pref(p.B));
+    int *s_cpref = reinterpret_cast<int *>(smem + M::cpref(p.B));
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int B = p.B, Hkv = p.Hkv;
@@ -441,18 +474,18 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
         }
     }
     __syncthreads();
-    if (warp == 0) tile_prefix(s_tiles, s_pref, B, Hkv, lane);
+    if (warp == 0) tile_prefix(s_tiles, s_pref, s_cpref, B, Hkv, lane);
     __syncthreads();
 
     grid_launch_dependents();  // the next grid may be placed (it waits for this one)
 
-    // ---- this warp's share of the global tile sequence
-    const int total = s_pref[B];
+    // ---- this warp's share of the global tile sequence (cut in cost space)
+    const int total = s_pref[B], TC = s_cpref[B];
     const int W = active_warps(p, total);
     const int w = blockIdx.x * NW + warp;
     if (w >= W) return;
-    const int t_begin = static_cast<int>(static_cast<int64_t>(w) * total / W);
-    const int t_end = static_cast<int>(static_cast<int64_t>(w + 1) * total / W);
+    const int t_begin = cost_to_tile(static_cast<int64_t>(w) * TC / W, s_tiles, s_pref, s_cpref, B);
+    const int t_end = cost_to_tile(static_cast<int64_t>(w + 1) * TC / W, s_tiles, s_pref, s_cpref, B);
     if (t_begin >= t_end) return;  // no CTA-wide barrier follows
 
     // barriers: [warp][stage][K, V] "tile half landed"
@@ -832,9 +865,8 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
                                               [](float2 a, float2 b) { return make_float2(a.x + b.x, a.y + b.y); });
             const int obase = halving_base<S::NO, S::OLEV>(lane, LPT);
             // the warps covering this context's global tiles [A, A + nt)
-            const int A = s_pref[r] + h * nt;
             int w_first, w_last;
-            context_warps(A, nt, W, total, w_first, w_last);
+            context_warps(s_cpref[r] + h * (nt + kCtxCost) + kCtxCost, nt, W, TC, w_first, w_last);
             float *out_rh = p.out + (static_cast<size_t>(r) * p.Hq + static_cast<size_t>(h) * G) * D;
             const bool whole = (w_first == w_last);
             float *slot = part_slot<D, G>(p, w, r * Hkv + h);
@@ -914,8 +946,6 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
     }
 }
 
-
-
 // ------------------------------------------------------------ combine grid
 // Log-sum-exp merge for GridCombine group sizes: one warp per (context,
 // query head of the group). All segments' (max, sum) pairs come in one load
@@ -933,6 +963,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const Param
     extern __shared__ __align__(16) int csm[];
     int *s_tiles = csm;
     int *s_pref = csm + p.B;
+    int *s_cpref = s_pref + p.B + 1;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int B = p.B, Hkv = p.Hkv;
 
@@ -943,9 +974,9 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const Param
         s_tiles[i] = ctx_ok(p, c) ? (c + TT - 1) / TT : 0;
     }
     __syncthreads();
-    if (warp == 0) tile_prefix(s_tiles, s_pref, B, Hkv, lane);
+    if (warp == 0) tile_prefix(s_tiles, s_pref, s_cpref, B, Hkv, lane);
     __syncthreads();
-    const int total = s_pref[B];
+    const int total = s_pref[B], TC = s_cpref[B];
     const int W = active_warps(p, total);
 
     grid_dependency_wait();  // the partials are complete and visible
@@ -958,7 +989,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const Param
         const int nt = s_tiles[r];
         if (nt == 0) continue;
         int w_first, w_last;
-        context_warps(s_pref[r] + h * nt, nt, W, total, w_first, w_last);
+        context_warps(s_cpref[r] + h * (nt + kCtxCost) + kCtxCost, nt, W, TC, w_first, w_last);
         if (w_first == w_last) continue;  // written by the decode grid itself
         const int nseg = w_last - w_first + 1;
         const float *base = part_slot<D, G>(p, w_first, rh);
@@ -1091,7 +1122,7 @@ static int launch(const Params &p, bool bf16, int blocks, cudaStream_t s)
     if constexpr (GridCombine<G>::value) {
         const int tasks = p.B * p.Hkv * G;
         const int cblocks = max(1, min((tasks + kCombineWarps - 1) / kCombineWarps, 4 * blocks));
-        const size_t csmem = align_up(sizeof(int) * (2 * static_cast<size_t>(p.B) + 1), 16);
+        const size_t csmem = align_up(sizeof(int) * (3 * static_cast<size_t>(p.B) + 2), 16);
         rc = check_cuda(launch_pdl(combine_kernel<D, G>, dim3(cblocks), dim3(kCombineWarps * 32), csmem, s, p),
                         "decode combine launch");
     }
