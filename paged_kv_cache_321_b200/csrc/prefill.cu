@@ -9,22 +9,28 @@
 //
 // B200 design. Prefill is a dense contraction (S = Q K^T and O = P V over
 // 128-key tiles), so it runs on the 5th-generation tensor cores:
-//  * one CTA per (sequence, kv head, 128/G query tokens): its 128 rows are
+//  * one CTA per (sequence, kv head, 128/G query tokens), launched longest
+//    first (a counting sort of the work items in every CTA's prologue): its
+//    128 rows are
 //    (query token, query head of the GQA group) pairs sharing the kv head's
 //    K and V, so one M=128 MMA serves the whole group;
-//  * warp 5 (one thread) streams K and V tiles of 128 keys with tiled TMA
+//  * warps 9 and 10 stream K and V tiles of 128 keys with tiled TMA
 //    copies (cp.async.bulk.tensor, no multicast) straight out of the block
 //    pool through a tensor map over [blocks*Hkv][block_size][D]; the block
 //    table supplies the third coordinate, the 128-byte swizzle produces the
 //    canonical UMMA operand layout;
-//  * warp 4 (one thread) issues tcgen05.mma kind::f16 (fp16 operands, fp32
+//  * warp 8 (one thread) issues tcgen05.mma kind::f16 (fp16 operands, fp32
 //    accumulation in TMEM): S(j) into one of two TMEM buffers while the
 //    softmax warps work on S(j-1), then O += P(j-1) V(j-1) into a TMEM
 //    accumulator;
-//  * warps 0-3 own one row each: tcgen05.ld of the S row, causal mask,
+//  * warps 0-7 own half a row each (two warps per 32-row TMEM quarter, one
+//    per 64-column half; row max and sum exchanged through shared memory):
+//    tcgen05.ld of the S row half, causal mask,
 //    online softmax with a lazily moved reference max (O in TMEM is rescaled
 //    only when a row max grows by more than 2^8), P rounded to fp16 and
-//    written swizzled to shared memory as the A operand of the PV MMA;
+//    written swizzled to shared memory as the A operand of the PV MMA. P is
+//    double-buffered, so the softmax of tile j runs while the tensor core
+//    does PV(j-1) and QK(j+1); it waits for PV(j-1) only to rescale O;
 //  * the epilogue reads O from TMEM, divides by the row sum and writes fp32.
 #include <cuda.h>
 
@@ -41,7 +47,9 @@ constexpr int D = 128;       // head dim of this kernel
 constexpr int BM = 128;      // rows per CTA: (query token, group head) pairs
 constexpr int BN = 128;      // keys per KV tile
 constexpr int NSTAGE = 2;    // K/V stages
-constexpr int NTHREADS = 192;
+constexpr int NSMX = 8;                       // softmax warps: two per 32-row quarter (one per 64-column half)
+constexpr int MMA_WARP = NSMX, K_WARP = NSMX + 1, V_WARP = NSMX + 2;  // MMA issuer, K and V producers
+constexpr int NTHREADS = (NSMX + 3) * 32;
 constexpr float kLazy = 8.0f;
 
 // shared-memory layout (bytes from a 1024-aligned base)
@@ -50,22 +58,26 @@ constexpr int TILE_BYTES = 2 * HALF_BYTES;       // 128 rows x 128 fp16
 constexpr int Q_OFF = 0;
 constexpr int K_OFF = Q_OFF + TILE_BYTES;
 constexpr int V_OFF = K_OFF + NSTAGE * TILE_BYTES;
-constexpr int P_OFF = V_OFF + NSTAGE * TILE_BYTES;
-constexpr int BAR_OFF = P_OFF + TILE_BYTES;
+constexpr int P_OFF = V_OFF + NSTAGE * TILE_BYTES;  // [2] P buffers: tile j uses P_OFF + (j & 1) * TILE_BYTES
+constexpr int BAR_OFF = P_OFF + 2 * TILE_BYTES;
 // barriers
 enum {
     B_KFULL = 0,             // [NSTAGE] K tile landed (TMA tx)
     B_VFULL = B_KFULL + 2,   // [NSTAGE] V tile landed
-    B_KVEMPTY = B_VFULL + 2, // [NSTAGE] stage free (PV of the tile done)
-    B_SFULL = B_KVEMPTY + 2, // [2] S buffer computed
-    B_SFREE = B_SFULL + 2,   // [2] S buffer read by the 4 softmax warps
-    B_PFULL = B_SFREE + 2,   // P written by the 4 softmax warps
-    B_ODONE = B_PFULL + 1,   // PV done (O stable, P free)
-    B_QFULL = B_ODONE + 1,   // Q written by the 4 softmax warps
-    NBARS = B_QFULL + 1
+    B_KEMPTY = B_VFULL + 2,  // [NSTAGE] K stage free (QK of the tile done)
+    B_VEMPTY = B_KEMPTY + 2, // [NSTAGE] V stage free (PV of the tile done)
+    B_SFULL = B_VEMPTY + 2,  // [2] S buffer computed
+    B_SFREE = B_SFULL + 2,   // [2] S buffer read by the softmax warps
+    B_PFULL = B_SFREE + 2,   // [2] P buffer written by the softmax warps
+    B_ODONE = B_PFULL + 2,   // [2] PV of tile j done (j & 1): O holds it, P buffer j & 1 is free
+    B_QFULL = B_ODONE + 2,   // Q written by the softmax warps
+    B_XCH = B_QFULL + 1,     // [4 quarters][2] row max (last: row sum) of both halves of a row published
+    NBARS = B_XCH + 8
 };
 constexpr int TMEM_PTR_OFF = BAR_OFF + NBARS * 8;
-constexpr int SMEM_BYTES = TMEM_PTR_OFF + 16 + 1024;  // + alignment slack
+constexpr int XCH_OFF = TMEM_PTR_OFF + 16;          // float [2 parities][2 halves][128 rows]
+constexpr int SMEM_BYTES = XCH_OFF + 2 * 2 * BM * 4;  // the dynamic region is 1024-aligned
+static_assert(SMEM_BYTES <= 227 * 1024, "prefill shared memory");
 constexpr uint32_t TMEM_COLS = 512;                    // S0, S1, O (128 columns each)
 
 struct Params {
@@ -76,6 +88,7 @@ struct Params {
     const int32_t *bt;      // [S][mbps]
     int *status;
     int S, Hq, Hkv, G, mbps, bs, num_blocks, max_seq_len, ntq;  // ntq: query tiles per sequence (grid)
+    int nbins;              // cost bins: KV tiles an item can read, 0 .. max_seq_len / BN + 1
     float qscale;           // softmax scale * log2(e), folded into Q
 };
 
@@ -202,9 +215,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v, const Params p)
 {
     constexpr int TQ = BM / G;  // query tokens per CTA
-    extern __shared__ unsigned char smem_raw[];
-    const uint32_t raw = smem_addr(smem_raw);
-    unsigned char *smem = smem_raw + ((1024 - (raw & 1023)) & 1023);
+    extern __shared__ __align__(1024) unsigned char smem[];
     const uint32_t sbase = smem_addr(smem);
     auto bar = [&](int i) { return sbase + BAR_OFF + i * 8; };
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(smem + TMEM_PTR_OFF);
@@ -214,8 +225,73 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // the previous grid has completed
     grid_dependency_wait();
     grid_launch_dependents();
-    // blockIdx: x = query tile (largest first), y = kv head, z = sequence
-    const int s = blockIdx.z, h = blockIdx.y, qt = p.ntq - 1 - blockIdx.x;
+    // ---- longest-first work order. Items are (sequence, query tile); an
+    // item's cost is the number of KV tiles it reads (0 for query tiles past
+    // its sequence's chunk and for sequences in error). The CTA launched
+    // L-th takes the unit of rank L in descending cost (ties by item index,
+    // kv heads innermost), so the longest items start first and the short
+    // ones fill the tail. Every CTA computes the same order: a counting sort
+    // of the item costs in shared memory (the P buffers are not in use yet).
+    int s, h, qt;
+    {
+        int *hist = reinterpret_cast<int *>(smem + P_OFF);
+        int *pick = reinterpret_cast<int *>(smem + XCH_OFF);
+        const int nitems = p.S * p.ntq;
+        auto cost = [&](int i) -> int {
+            const int si = i / p.ntq, t0i = (i - si * p.ntq) * TQ;
+            const int ql = p.cu_q[si + 1] - p.cu_q[si], c = p.ctx[si];
+            if (t0i >= ql || ql <= 0 || c < ql || c > p.mbps * p.bs || c > p.max_seq_len) return 0;
+            return (c - ql + min(ql, t0i + TQ) - 1) / BN + 1;
+        };
+        for (int i = tid; i < p.nbins; i += NTHREADS) hist[i] = 0;
+        __syncthreads();
+        for (int i = tid; i < nitems; i += NTHREADS) atomicAdd(&hist[cost(i)], 1);
+        __syncthreads();
+        if (warp == 0) {
+            const int R = blockIdx.x / p.Hkv;  // rank of this CTA's item
+            // the cost bin holding rank R, scanning bins from the most costly
+            int above = 0, bin = 0;
+            for (int top = p.nbins - 1; top >= 0; top -= 32) {
+                const int v = top - lane;
+                const int n = v >= 0 ? hist[v] : 0;
+                int x = n;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, x, off);
+                    if (lane >= off) x += y;
+                }
+                const unsigned hit = __ballot_sync(0xffffffffu, n > 0 && above + x - n <= R && R < above + x);
+                if (hit) {
+                    const int src = __ffs(hit) - 1;
+                    bin = top - src;
+                    above += __shfl_sync(0xffffffffu, x - n, src);
+                    break;
+                }
+                above += __shfl_sync(0xffffffffu, x, 31);
+            }
+            // the (R - above)-th item of that cost, in index order
+            int k = R - above, item = 0;
+            for (int base = 0; base < nitems; base += 32) {
+                const int i = base + lane;
+                const unsigned m = __ballot_sync(0xffffffffu, i < nitems && cost(i) == bin);
+                const int c = __popc(m);
+                if (k < c) {
+                    unsigned mm = m;
+                    for (int q = 0; q < k; ++q) mm &= mm - 1;  // drop the k lowest matches
+                    item = base + __ffs(mm) - 1;
+                    break;
+                }
+                k -= c;
+            }
+            if (lane == 0) pick[0] = item;
+        }
+        __syncthreads();
+        const int item = pick[0];
+        s = item / p.ntq;
+        qt = item - s * p.ntq;
+        h = blockIdx.x - (blockIdx.x / p.Hkv) * p.Hkv;
+        __syncthreads();  // pick and hist are reused below
+    }
     const int q0 = p.cu_q[s], q_len = p.cu_q[s + 1] - q0;
     const int ctx = p.ctx[s];
     const int t0 = qt * TQ;  // first query token of this tile (within the sequence)
@@ -225,18 +301,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (qt == 0 && h == 0 && tid == 0) report(p.status, KVP_ERANGE, s);
         return;  // uniform for the CTA: nothing allocated yet
     }
+    if (sbase & 1023) {  // the 128-byte swizzle atoms need a 1024-aligned region
+        if (tid == 0) report(p.status, KVP_EUNSUPPORTED, -1);
+        return;  // uniform for the CTA: nothing allocated yet
+    }
     const int first_pos = ctx - q_len;                   // position of query 0
     const int last_pos = first_pos + min(q_len, t0 + TQ) - 1;
     const int nkv = last_pos / BN + 1;                   // KV tiles this CTA reads
 
     if (tid == 0) {
         for (int i = 0; i < NBARS; ++i) {
-            const bool by_softmax_warps = i == B_SFREE || i == B_SFREE + 1 || i == B_PFULL || i == B_QFULL;
-            mbar_init(bar(i), by_softmax_warps ? 4 : 1);
+            const bool by_softmax_warps =
+                i == B_SFREE || i == B_SFREE + 1 || i == B_PFULL || i == B_PFULL + 1 || i == B_QFULL;
+            mbar_init(bar(i), by_softmax_warps ? NSMX : (i >= B_XCH ? 2 : 1));
         }
         mbar_init_fence();
     }
-    if (warp == 4) {
+    if (warp == MMA_WARP) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tmem_ptr)),
                      "r"(TMEM_COLS));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -247,49 +328,56 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t tmem = *tmem_ptr;
     bool timed_out = false;
 
-    if (warp == 5) {
-        // ------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            const int32_t *btr = p.bt + static_cast<size_t>(s) * p.mbps;
-            const uint32_t half_rows_bytes = p.bs * 128;  // one block's rows of one 64-column half
-            for (int j = 0; j < nkv && !timed_out; ++j) {
-                const int st = j % NSTAGE;
-                if (j >= NSTAGE && !mbar_wait_bounded(bar(B_KVEMPTY + st), ((j / NSTAGE) - 1) & 1)) {
+    if (warp == K_WARP || warp == V_WARP) {
+        // ------------------------------------------------- TMA producers (K, V)
+        // One warp streams K tiles, another V tiles, each gated only by its
+        // own stage-free barrier: K of stage st is free once QK of tile
+        // j - NSTAGE is done, V once its PV is, so K runs ahead of the
+        // softmax and QK(j + 1) overlaps the softmax of tile j. Lane b handles
+        // block b of each 128-key tile (at most 8 blocks: the block size is at
+        // least 16): the block ids of a tile come in one batch of loads (the
+        // next tile's while this one's copies fly), and each lane issues its
+        // own block's copies.
+        const int kv = warp == V_WARP;
+        const int32_t *btr = p.bt + static_cast<size_t>(s) * p.mbps;
+        const uint32_t half_rows_bytes = p.bs * 128;  // one block's rows of one 64-column half
+        auto block_of = [&](int j) {
+            const int first = (j * BN) / p.bs;
+            const int nblk = (min(BN, ctx - j * BN) + p.bs - 1) / p.bs;
+            return lane < nblk ? btr[first + lane] : -1;
+        };
+        int blk = block_of(0);
+        for (int j = 0; j < nkv && !timed_out; ++j) {
+            const int st = j % NSTAGE;
+            const int nblk = (min(BN, ctx - j * BN) + p.bs - 1) / p.bs;
+            const bool mine = lane < nblk;
+            const bool valid = mine && blk >= 0 && blk < p.num_blocks;
+            if (mine && !valid && !kv) report(p.status, KVP_ERANGE, s);
+            const int loaded = __popc(__ballot_sync(0xffffffffu, valid));
+            const uint32_t bytes = static_cast<uint32_t>(loaded) * 2 * half_rows_bytes;
+            if (j >= NSTAGE) {
+                bool ok = true;
+                if (lane == 0) ok = mbar_wait_bounded(bar((kv ? B_VEMPTY : B_KEMPTY) + st), ((j / NSTAGE) - 1) & 1);
+                if (!__shfl_sync(0xffffffffu, ok, 0)) {
                     timed_out = true;
                     break;
                 }
-                // blocks holding keys [j*BN, min(ctx, (j+1)*BN))
-                const int nkeys = min(BN, ctx - j * BN);
-                const int nblk = (nkeys + p.bs - 1) / p.bs;
-                int loaded = 0;
-                for (int b = 0; b < nblk; ++b) {
-                    const int blk = btr[(j * BN) / p.bs + b];
-                    if (blk >= 0 && blk < p.num_blocks) ++loaded;
-                }
-                const uint32_t bytes = static_cast<uint32_t>(loaded) * 2 * half_rows_bytes;
-                if (bytes) {
-                    mbar_arrive_expect_tx(bar(B_KFULL + st), bytes);
-                    mbar_arrive_expect_tx(bar(B_VFULL + st), bytes);
-                } else {
-                    mbar_arrive(bar(B_KFULL + st));
-                    mbar_arrive(bar(B_VFULL + st));
-                }
-                for (int b = 0; b < nblk; ++b) {
-                    const int blk = btr[(j * BN) / p.bs + b];
-                    if (blk < 0 || blk >= p.num_blocks) {
-                        report(p.status, KVP_ERANGE, s);
-                        continue;
-                    }
-                    const int tile = blk * p.Hkv + h;
-                    for (int hf = 0; hf < 2; ++hf) {
-                        const uint32_t off = hf * HALF_BYTES + b * half_rows_bytes;
-                        tma_load_3d(sbase + K_OFF + st * TILE_BYTES + off, &tmap_k, hf * 64, 0, tile, bar(B_KFULL + st));
-                        tma_load_3d(sbase + V_OFF + st * TILE_BYTES + off, &tmap_v, hf * 64, 0, tile, bar(B_VFULL + st));
-                    }
-                }
             }
+            const uint32_t full = bar((kv ? B_VFULL : B_KFULL) + st);
+            if (lane == 0) {
+                if (bytes) mbar_arrive_expect_tx(full, bytes);
+                else mbar_arrive(full);
+            }
+            __syncwarp();
+            if (valid) {
+                const int tile = blk * p.Hkv + h;
+                const uint32_t dst0 = sbase + (kv ? V_OFF : K_OFF) + st * TILE_BYTES + lane * half_rows_bytes;
+                for (int hf = 0; hf < 2; ++hf)
+                    tma_load_3d(dst0 + hf * HALF_BYTES, kv ? &tmap_v : &tmap_k, hf * 64, 0, tile, full);
+            }
+            if (j + 1 < nkv) blk = block_of(j + 1);
         }
-    } else if (warp == 4) {
+    } else if (warp == MMA_WARP) {
         // ------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t IDS = idesc_f16(BM, BN, BF16, false);  // S = Q K^T
@@ -305,21 +393,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                             sdesc(sbase + K_OFF + st * TILE_BYTES + koff, 16, 1024), IDS, kk > 0);
                 }
                 mma_commit(bar(B_SFULL + b));
+                mma_commit(bar(B_KEMPTY + st));
                 return true;
             };
             auto pv = [&](int j) -> bool {
-                const int st = j % NSTAGE;
-                if (!mbar_wait_bounded(bar(B_PFULL), j & 1)) return false;
+                const int st = j % NSTAGE, pb = j & 1;
+                if (!mbar_wait_bounded(bar(B_PFULL + pb), (j >> 1) & 1)) return false;
                 if (!mbar_wait_bounded(bar(B_VFULL + st), (j / NSTAGE) & 1)) return false;
                 tc_fence_after();
                 for (int kk = 0; kk < BN / 16; ++kk) {
                     const uint32_t aoff = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;  // P: keys are K
                     const uint32_t boff = kk * 16 * 128;                              // V: 16 key rows
-                    mma_f16(tmem + 256, sdesc(sbase + P_OFF + aoff, 16, 1024),
+                    mma_f16(tmem + 256, sdesc(sbase + P_OFF + pb * TILE_BYTES + aoff, 16, 1024),
                             sdesc(sbase + V_OFF + st * TILE_BYTES + boff, HALF_BYTES, 1024), IDO, j > 0 || kk > 0);
                 }
-                mma_commit(bar(B_ODONE));
-                mma_commit(bar(B_KVEMPTY + st));
+                mma_commit(bar(B_ODONE + pb));
+                mma_commit(bar(B_VEMPTY + st));
                 return true;
             };
             bool ok = mbar_wait_bounded(bar(B_QFULL), 0);
@@ -332,17 +421,33 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
     } else {
         // ------------------------------------------------------ softmax warps
-        const int r = tid;  // row = g * TQ + t
+        // Warp w owns rows r = 32*(w%4) + lane (its TMEM lanes) and columns
+        // 64*(w/4) .. +63 of them; the two warps of a row exchange the row
+        // max (and at the end the row sum) through shared memory, ordered by
+        // a 2-arrival mbarrier per quarter and tile parity.
+        const int qw = warp & 3, hf = warp >> 2;
+        const int r = qw * 32 + lane;  // row = g * TQ + t
         const int g = r / TQ, t = r % TQ;
         const int qi = t0 + t;  // query index in the sequence
         const bool row_ok = qi < q_len;
         const int pos = row_ok ? first_pos + qi : -1;  // sees keys 0..pos
         const size_t qrow = (static_cast<size_t>(q0 + qi) * p.Hq + static_cast<size_t>(h) * G + g) * D;
-        // Q row: scale, round to 16 bits, store swizzled (two 64-column halves)
+        float *xch = reinterpret_cast<float *>(smem + XCH_OFF);  // [parity][half][row]
+        // publishes v for this row and returns the partner half's value for
+        // exchange round k (k = tile index; the final sums use k = nkv)
+        auto exchange = [&](int k, float v, float &other) -> bool {
+            xch[((k & 1) * 2 + hf) * BM + r] = v;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_XCH + qw * 2 + (k & 1)));
+            if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar(B_XCH + qw * 2 + (k & 1)), (k >> 1) & 1))) return false;
+            other = xch[((k & 1) * 2 + (hf ^ 1)) * BM + r];
+            return true;
+        };
+        // Q row half: scale, round to 16 bits, store swizzled
         {
-            const float4 *src = reinterpret_cast<const float4 *>(p.q + qrow);
-#pragma unroll 4
-            for (int c = 0; c < 16; ++c) {  // 16 chunks of 8 values
+            const float4 *src = reinterpret_cast<const float4 *>(p.q + qrow) + hf * 16;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {  // 8 chunks of 8 values
                 float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b4 = a;
                 if (row_ok) {
                     a = src[2 * c];
@@ -351,14 +456,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const float sc = p.qscale;
                 const uint4 w = make_uint4(pack2<BF16>(a.x * sc, a.y * sc), pack2<BF16>(a.z * sc, a.w * sc),
                                            pack2<BF16>(b4.x * sc, b4.y * sc), pack2<BF16>(b4.z * sc, b4.w * sc));
-                *reinterpret_cast<uint4 *>(smem + Q_OFF + (c >> 3) * HALF_BYTES + swz(r, c & 7)) = w;
+                *reinterpret_cast<uint4 *>(smem + Q_OFF + hf * HALF_BYTES + swz(r, c)) = w;
             }
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_QFULL));
 
-        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        const uint32_t lane_base = static_cast<uint32_t>(qw * 32) << 16;
+        const uint32_t col0 = hf * 64;  // this warp's first column of S and O
         float m_ref = -INFINITY, l = 0.0f;
         for (int j = 0; j < nkv && !timed_out; ++j) {
             const int b = j & 1;
@@ -367,11 +473,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 break;
             }
             tc_fence_after();
-            float sv[BN];
+            float sv[64];
 #pragma unroll
-            for (int c = 0; c < BN / 32; ++c) {
+            for (int c = 0; c < 2; ++c) {
                 float tmp[32];
-                tmem_ld32(tmem + lane_base + b * 128 + c * 32, tmp);
+                tmem_ld32(tmem + lane_base + b * 128 + col0 + c * 32, tmp);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) sv[c * 32 + i] = tmp[i];
             }
@@ -379,31 +485,45 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_SFREE + b));
-            // causal mask and row max
-            const int key0 = j * BN;
+            // causal mask and row max (this half, then both)
+            const int key0 = j * BN + col0;
             float mx = -INFINITY;
 #pragma unroll
-            for (int i = 0; i < BN; ++i) {
+            for (int i = 0; i < 64; ++i) {
                 if (key0 + i > pos) sv[i] = -INFINITY;
                 mx = fmaxf(mx, sv[i]);
             }
-            // PV of the previous tile must be done before P is rewritten and O rescaled
-            if (j > 0 && !__all_sync(0xffffffffu, mbar_wait_bounded(bar(B_ODONE), (j - 1) & 1))) {
+            float mo;
+            if (!exchange(j, mx, mo)) {
+                timed_out = true;
+                break;
+            }
+            mx = fmaxf(mx, mo);
+            // O may be rescaled only once the PV of the previous tile is in it
+            // (rare: the reference max moves lazily); P buffer j & 1 is free
+            // once the PV of tile j - 2 is done. Otherwise this tile's
+            // softmax overlaps the tensor core's PV(j - 1) and QK(j + 1).
+            const bool move = mx > m_ref + kLazy;  // the same in both halves of a row
+            const bool rescale = __any_sync(0xffffffffu, move) && j > 0;
+            if (rescale && !__all_sync(0xffffffffu, mbar_wait_bounded(bar(B_ODONE + ((j - 1) & 1)), ((j - 1) >> 1) & 1))) {
+                timed_out = true;
+                break;
+            }
+            if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait_bounded(bar(B_ODONE + (j & 1)), ((j - 2) >> 1) & 1))) {
                 timed_out = true;
                 break;
             }
             tc_fence_after();
-            const bool move = mx > m_ref + kLazy;
-            if (__any_sync(0xffffffffu, move) && j > 0) {
+            if (rescale) {
                 const float alpha = move ? ex2(m_ref - mx) : 1.0f;
 #pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
+                for (int c = 0; c < 2; ++c) {
                     float o[32];
-                    tmem_ld32(tmem + lane_base + 256 + c * 32, o);
+                    tmem_ld32(tmem + lane_base + 256 + col0 + c * 32, o);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) o[i] *= alpha;
-                    tmem_st32(tmem + lane_base + 256 + c * 32, o);
+                    tmem_st32(tmem + lane_base + 256 + col0 + c * 32, o);
                 }
                 tmem_wait_st();
                 l *= alpha;
@@ -411,7 +531,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (move) m_ref = mx;
             // P = exp2(s - m_ref) rounded to 16 bits; l sums the rounded values
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
+            for (int c = 0; c < 8; ++c) {
                 uint32_t w[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -422,12 +542,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     const float2 back = unpack<BF16>(w[e]);
                     l += back.x + back.y;
                 }
-                *reinterpret_cast<uint4 *>(smem + P_OFF + (c >> 3) * HALF_BYTES + swz(r, c & 7)) =
+                *reinterpret_cast<uint4 *>(smem + P_OFF + (j & 1) * TILE_BYTES + hf * HALF_BYTES + swz(r, c)) =
                     make_uint4(w[0], w[1], w[2], w[3]);
             }
             // keys of this tile past the context: their V rows may hold
             // anything (or were not loaded); zero them so 0 * V stays 0
-            const int nkeys = min(BN, ctx - key0);
+            const int nkeys = min(BN, ctx - j * BN);
             if (nkeys < BN) {
                 const int st = j % NSTAGE;
                 if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar(B_VFULL + st), (j / NSTAGE) & 1))) {
@@ -435,7 +555,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     break;
                 }
                 unsigned char *vt = smem + V_OFF + st * TILE_BYTES;
-                for (int idx = r; idx < (BN - nkeys) * 16; idx += 128) {
+                for (int idx = r + hf * BM; idx < (BN - nkeys) * 16; idx += 2 * BM) {
                     const int row = nkeys + idx / 16, chunk = idx % 16;
                     *reinterpret_cast<uint4 *>(vt + (chunk >> 3) * HALF_BYTES + row * 128 + ((chunk & 7) << 4)) =
                         make_uint4(0u, 0u, 0u, 0u);
@@ -444,17 +564,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_PFULL));
+            if (lane == 0) mbar_arrive(bar(B_PFULL + (j & 1)));
         }
-        // epilogue: O / l
-        if (!timed_out && __all_sync(0xffffffffu, mbar_wait_bounded(bar(B_ODONE), (nkv - 1) & 1))) {
+        // epilogue: O / (sum of both halves' l)
+        float lo = 0.0f;
+        if (!timed_out && exchange(nkv, l, lo) &&
+            __all_sync(0xffffffffu, mbar_wait_bounded(bar(B_ODONE + ((nkv - 1) & 1)), ((nkv - 1) >> 1) & 1))) {
             tc_fence_after();
-            const float inv = l > 0.0f ? 1.0f / l : 0.0f;
-            float4 *dst = reinterpret_cast<float4 *>(p.out + qrow);
+            const float lt = l + lo;
+            const float inv = lt > 0.0f ? 1.0f / lt : 0.0f;
+            float4 *dst = reinterpret_cast<float4 *>(p.out + qrow) + hf * 16;
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = 0; c < 2; ++c) {
                 float o[32];
-                tmem_ld32(tmem + lane_base + 256 + c * 32, o);
+                tmem_ld32(tmem + lane_base + 256 + col0 + c * 32, o);
                 tmem_wait_ld();
                 if (row_ok) {
 #pragma unroll
@@ -470,7 +593,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 4) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+    if (warp == MMA_WARP)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
 }
 
 // ------------------------------------------------------------------- host
@@ -520,7 +644,10 @@ static int launch(const CUtensorMap &mk, const CUtensorMap &mv, const Params &p,
     int rc = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES),
                         "prefill smem attribute");
     if (rc) return rc;
-    return check_cuda(launch_pdl(kern, dim3(p.ntq, p.Hkv, p.S), dim3(NTHREADS), SMEM_BYTES, s, mk, mv, p),
+    const int64_t units = static_cast<int64_t>(p.ntq) * p.Hkv * p.S;
+    if (units > 0x7FFFFFFF) return set_error(KVP_EINVAL, "prefill: too many query tiles");
+    if (static_cast<int64_t>(p.nbins) * 4 > TILE_BYTES * 2) return set_error(KVP_EUNSUPPORTED, "prefill: max_seq_len too large");
+    return check_cuda(launch_pdl(kern, dim3(static_cast<unsigned>(units)), dim3(NTHREADS), SMEM_BYTES, s, mk, mv, p),
                       "prefill launch");
 }
 
@@ -565,6 +692,7 @@ extern "C" int paged_prefill_attention(kvp_pool *pool, int layer, const kvp_attn
     p.q = q, p.out = out, p.cu_q = cu_q, p.ctx = ctx_lens, p.bt = block_tables, p.status = pool->status;
     p.S = S, p.Hq = Hq, p.Hkv = Hkv, p.G = G, p.mbps = max_blocks_per_seq, p.bs = bs;
     p.num_blocks = pool->cfg.num_blocks, p.max_seq_len = pool->cfg.max_seq_len;
+    p.nbins = pool->cfg.max_seq_len / pre::BN + 2;
     const double scale = static_cast<double>(static_cast<float>(1.0 / sqrt(static_cast<double>(pre::D))));
     p.qscale = static_cast<float>(scale * 1.4426950408889634);
     const bool bf16 = pool->cfg.kv_dtype == KVP_BF16;
@@ -572,7 +700,6 @@ extern "C" int paged_prefill_attention(kvp_pool *pool, int layer, const kvp_attn
     auto go = [&](auto g_tag) -> int {
         constexpr int GG = decltype(g_tag)::value;
         p.ntq = (max_q_len + pre::BM / GG - 1) / (pre::BM / GG);
-        if (p.ntq > 65535) return set_error(KVP_EINVAL, "max_q_len too large");
         return bf16 ? pre::launch<GG, true>(mk, mv, p, s) : pre::launch<GG, false>(mk, mv, p, s);
     };
     switch (G) {
