@@ -192,8 +192,11 @@ size_t paged_decode_workspace_size(const kvp_pool *pool, const kvp_attn_config *
  * accumulated in fp32 with an online softmax over 16-key tiles. The tiles of
  * all (sequence, kv head) contexts are divided evenly among the GPU's warps;
  * a context shared by several warps is combined from their (max, sum,
- * unnormalised output) partials by log-sum-exp in fp32 by the last of them to
- * finish. split_tokens is the fewest keys one warp takes (0 = automatic;
+ * unnormalised output) partials by log-sum-exp in fp32 (by the last of them
+ * to finish, or by a second small grid). With 4 or 8 query heads per kv head
+ * and block_size >= 16 the tile products run on tensor cores with 16-bit
+ * inputs: K and V exactly, q and the softmax weights each as a 16-bit high
+ * part plus the 16-bit rounding of the remainder (about 16 more bits). split_tokens is the fewest keys one warp takes (0 = automatic;
  * otherwise a multiple of 16): a large value keeps each context on one warp.
  *
  *   q, out        [B][Hq][D] float32

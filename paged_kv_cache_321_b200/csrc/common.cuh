@@ -3,6 +3,7 @@
 // conversion) used by the kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
 #include <cuda_bf16.h>
@@ -28,6 +29,11 @@ int check_pool(const kvp_pool *pool, int layer);
 int resolve_attn(const kvp_pool *pool, const kvp_attn_config *attn, int *Hq, int *Hkv, int *G);
 
 inline bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+// Tensor map over one layer's K or V pool viewed as [blocks*Hkv][bs][D] 16-bit
+// words, with a box of 64 columns x box_rows rows x 1 (block, head) tile and
+// the 128-byte swizzle (the canonical layout of a 128-byte-row operand).
+int make_pool_tmap(CUtensorMap *map, const uint16_t *base, const kvp_pool *pool, int box_rows);
 
 // --------------------------------------------------------------- device side
 constexpr int kWaitLimitNs = 1000 * 1000 * 1000;  // 1 s bound on any wait

@@ -1,5 +1,9 @@
 // paged_decode_attention: one query token per sequence, GQA attention over a
 // block-pooled KV cache, split over the context with a log-sum-exp combine.
+// Two kernels share the work distribution below: decode_kernel computes on
+// CUDA cores (any group size and block size), decode_tc_kernel on tensor
+// cores (groups of 4 and 8 with blocks of at least 16 tokens; see its own
+// description further down).
 //
 // Method: the batch kernel of runHybridAttentionBlockBatch in
 // makarna/pkg/model/arch/hybrid_decoder.go (one query per request, per-request
@@ -946,6 +950,426 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
     }
 }
 
+
+// ------------------------------------- groups of 4 and 8 heads: tensor cores
+// With 4 or 8 query heads per kv head the per-tile arithmetic (2 x 16 tokens
+// x D x G multiply-adds, plus unpacking and lane reductions) costs the
+// CUDA-core kernel about as many issue slots as the memory system needs to
+// deliver the tile (8 heads: twice as many), so this variant does both
+// contractions of a tile with warp-level mma.sync (m16n8k16, 16-bit inputs,
+// fp32 accumulation); the rest of the design is unchanged (persistent,
+// stream-K in cost space, per-warp rings), the split partials go to the
+// merge grid:
+//  * S = Q K^T: A = the group's query heads (rows past the group and rows
+//    8..15 zero), B = the K tile as loaded; q is split into a 16-bit high
+//    part and the 16-bit rounding of the remainder, both multiplied, so the
+//    scores keep about 16 bits more than a 16-bit q would (K is exact);
+//  * the accumulator of S holds (head g, tokens 2q, 2q+1, 2q+8, 2q+9) in lane
+//    4g+q, which is exactly the B operand of O^T += V^T P^T: the online
+//    softmax runs in registers (quad shuffles for the row max and sum) and P
+//    feeds the PV product directly, again as high + low 16-bit parts whose
+//    sum is also what the row sum adds;
+//  * A of the PV product is V^T, read with ldmatrix.trans; K and V tiles come
+//    in as 64-column boxes of a tensor map with the 128-byte swizzle (three
+//    ring stages per warp), so all ldmatrix reads are free of bank conflicts;
+//  * O^T (D x 8 heads) stays in registers; the segment end writes the rows
+//    (or the partial) straight from the accumulator layout.
+template <int D>
+struct TcShape {
+    static constexpr int KC = D / 16;           // 16-wide chunks of the head dim
+    static constexpr int NH = D / 64;           // 64-column (128-byte) boxes per tile
+    static constexpr int BOX_BYTES = TT * 128;  // one box: 16 rows x 128 bytes
+    static constexpr int HALF_BYTES = NH * BOX_BYTES;  // K (or V) of one tile
+    static constexpr int STAGE_BYTES = 2 * HALF_BYTES;
+    static constexpr int NS = 3;                              // ring stages per warp
+    // the rings fill 192 KB of shared memory: deeper rings beat more warps
+    // (12 x 2 stages) except where many requests share blocks in L2
+    static constexpr int NW = (D <= 128 ? 12 : 6) * 2 / NS;
+    static_assert(D % 64 == 0, "head dim");
+};
+
+template <int D>
+struct TcSmem {
+    using S = TcShape<D>;
+    static constexpr size_t bars = static_cast<size_t>(S::NW) * S::NS * S::STAGE_BYTES;  // stages first (1024-aligned)
+    static constexpr size_t masks = bars + S::NW * S::NS * 2 * 8;
+    static constexpr size_t tiles = align_up(masks + S::NW * S::NS * 4, 16);
+    __host__ __device__ static size_t pref(int B) { return align_up(tiles + 4 * static_cast<size_t>(B), 16); }
+    __host__ __device__ static size_t cpref(int B) { return align_up(pref(B) + 4 * static_cast<size_t>(B + 1), 16); }
+    __host__ __device__ static size_t total(int B) { return align_up(cpref(B) + 4 * static_cast<size_t>(B + 1), 128); }
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4])
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4])
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+// d += A (16x16, row) * B (16x8, col); A rows 8..15 of the QK product are zero.
+template <bool BF16>
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1)
+{
+    if (BF16)
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+            "{%0,%1,%2,%3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    else
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+            "{%0,%1,%2,%3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// (hi, lo) 16-bit pairs of (x, y): hi = nearest 16-bit value, lo = nearest
+// 16-bit value of the remainder (computed exactly in fp32).
+template <bool BF16>
+__device__ __forceinline__ void split2(float x, float y, uint32_t &hi, uint32_t &lo)
+{
+    hi = cvt_pair<BF16>(x, y);
+    const float2 h = unpack2<BF16>(hi);
+    lo = cvt_pair<BF16>(x - h.x, y - h.y);
+}
+
+// Address of the 16-byte chunk (row, 8-element chunk c8 of the D columns) in
+// a K or V tile stored as NH swizzled 64-column boxes.
+template <int D>
+__device__ __forceinline__ uint32_t tc_addr(uint32_t tile, int row, int c8)
+{
+    return tile + (c8 >> 3) * TcShape<D>::BOX_BYTES + row * 128 + (((c8 & 7) ^ (row & 7)) << 4);
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int c0, int c1, int c2, uint32_t bar,
+                                            uint64_t pol)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar), "l"(pol)
+        : "memory");
+}
+
+template <int D, int G, bool BF16>
+__global__ void __launch_bounds__(TcShape<D>::NW * 32, 1)
+    decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+                     const Params p)
+{
+    static_assert(G == 4 || G == 8, "the MMA rows hold 8 heads: groups of 4 use half of them");
+    using S = TcShape<D>;
+    using M = TcSmem<D>;
+    constexpr int NW = S::NW, KC = S::KC, NH = S::NH, NST = S::NS;
+    extern __shared__ __align__(1024) unsigned char tc_smem[];
+    unsigned char *smem = tc_smem;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + M::bars);
+    int *nvalid_all = reinterpret_cast<int *>(smem + M::masks);
+    int *s_tiles = reinterpret_cast<int *>(smem + M::tiles);
+    int *s_pref = reinterpret_cast<int *>(smem + M::pref(p.B));
+    int *s_cpref = reinterpret_cast<int *>(smem + M::cpref(p.B));
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int B = p.B, Hkv = p.Hkv;
+    if (smem_addr(smem) & 1023) {  // the swizzled boxes need a 1024-aligned region
+        if (tid == 0) report(p.status, KVP_EUNSUPPORTED, -1);
+        return;  // uniform for the CTA, before any barrier
+    }
+
+    grid_dependency_wait();
+    {
+        const int64_t lines = (static_cast<int64_t>(B) * p.mbps * 4 + 127) / 128;
+        const int64_t lo = lines * blockIdx.x / gridDim.x, hi = lines * (blockIdx.x + 1) / gridDim.x;
+        const char *bt_bytes = reinterpret_cast<const char *>(p.bt);
+        for (int64_t l = lo + tid; l < hi && l < lo + 4 * NW * 32; l += NW * 32) prefetch_l2(bt_bytes + l * 128);
+    }
+    for (int i = tid; i < B; i += NW * 32) {
+        const int c = p.ctx[i];
+        const bool ok = ctx_ok(p, c);
+        s_tiles[i] = ok ? (c + TT - 1) / TT : 0;
+        if (blockIdx.x == 0 && (!ok || c == 0)) {
+            if (!ok) report(p.status, KVP_ERANGE, i);
+            float4 *o = reinterpret_cast<float4 *>(p.out + static_cast<size_t>(i) * p.Hq * D);
+            for (int k = 0; k < p.Hq * D / 4; ++k) o[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+    __syncthreads();
+    if (warp == 0) tile_prefix(s_tiles, s_pref, s_cpref, B, Hkv, lane);
+    __syncthreads();
+    grid_launch_dependents();
+
+    const int total = s_pref[B], TC = s_cpref[B];
+    const int W = active_warps(p, total);
+    const int w = blockIdx.x * NW + warp;
+    if (w >= W) return;
+    const int t_begin = cost_to_tile(static_cast<int64_t>(w) * TC / W, s_tiles, s_pref, s_cpref, B);
+    const int t_end = cost_to_tile(static_cast<int64_t>(w + 1) * TC / W, s_tiles, s_pref, s_cpref, B);
+    if (t_begin >= t_end) return;  // no CTA-wide barrier follows
+
+    const uint32_t kbar0 = smem_addr(&bars[warp * NST * 2]);
+    if (lane < 2 * NST) mbar_init(kbar0 + lane * 8, 1);
+    mbar_init_fence();
+    __syncwarp();
+
+    auto locate = [&](int t, Cursor &c) {
+        int lo = 0, hi = B;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (s_pref[mid] <= t) lo = mid;
+            else hi = mid;
+        }
+        c.t = t;
+        c.r = lo;
+        c.nt = s_tiles[lo];
+        const int local = t - s_pref[lo];
+        c.h = local / c.nt;
+        c.ti = local - c.h * c.nt;
+    };
+    auto advance = [&](Cursor &c) {
+        ++c.t;
+        if (++c.ti == c.nt) {
+            c.ti = 0;
+            if (++c.h == Hkv) {
+                c.h = 0;
+                do {
+                    ++c.r;
+                } while (c.r < B && s_tiles[c.r] == 0);
+                if (c.r < B) c.nt = s_tiles[c.r];
+            }
+        }
+    };
+
+    const uint32_t ring = smem_addr(smem) + warp * NST * S::STAGE_BYTES;
+    int *nvalid = nvalid_all + warp * NST;
+    const int ntile = t_end - t_begin;
+    const uint64_t l2pol = l2_evict_first_policy();
+
+    // copy descriptors of 32 consecutive tiles, one per lane: tensor
+    // coordinates (block * Hkv + head, first row in the block), valid
+    // tokens (0: block id outside the pool) and the segment's query row
+    int d_tile = 0, d_row = 0, d_nv = 0, d_q = -1, dbase = 0;
+    auto load_desc = [&](int base) {
+        dbase = base;
+        d_tile = d_row = d_nv = 0;
+        d_q = -1;
+        const int i = base + lane;
+        if (i < ntile) {
+            Cursor c;
+            locate(t_begin + i, c);
+            if (c.ti == 0 || i == 0) d_q = c.r * p.Hq + c.h * G;
+            const int ctx = p.ctx[c.r];
+            const int tb = c.ti * TT;
+            const int blk = p.bt[static_cast<size_t>(c.r) * p.mbps + tb / p.bs];
+            if (blk >= 0 && blk < p.num_blocks) {
+                d_tile = blk * Hkv + c.h;
+                d_row = tb % p.bs;
+                d_nv = min(TT, ctx - tb);
+            } else {
+                report(p.status, KVP_ERANGE, c.r);
+            }
+        }
+    };
+    auto issue = [&](int i, int half, int st) {
+        if (i - dbase >= 32) load_desc(i);
+        const int tile = __shfl_sync(0xffffffffu, d_tile, i - dbase);
+        const int row = __shfl_sync(0xffffffffu, d_row, i - dbase);
+        const int nv = __shfl_sync(0xffffffffu, d_nv, i - dbase);
+        if (half == 0) {
+            const int qrow = __shfl_sync(0xffffffffu, d_q, i - dbase);
+            if (qrow >= 0)
+                for (int l = lane; l < G * D / 32; l += 32) prefetch_l1(p.q + static_cast<size_t>(qrow) * D + l * 32);
+        }
+        if (lane == 0) {
+            fence_proxy_async_smem();
+            const uint32_t bar = kbar0 + (st * 2 + half) * 8;
+            if (nv > 0) {
+                mbar_arrive_expect_tx(bar, S::HALF_BYTES);
+                const uint32_t dst = ring + st * S::STAGE_BYTES + half * S::HALF_BYTES;
+                for (int hh = 0; hh < NH; ++hh)
+                    tma_load_3d(dst + hh * S::BOX_BYTES, half ? &tmap_v : &tmap_k, hh * 64, row, tile, bar, l2pol);
+            } else {
+                mbar_arrive(bar);
+            }
+            if (half == 0) nvalid[st] = nv;
+        }
+    };
+
+    load_desc(0);
+    for (int i = 0; i < NST && i < ntile; ++i) {
+        issue(i, 0, i);
+        issue(i, 1, i);
+    }
+    __syncwarp();
+
+    Cursor cons;
+    locate(t_begin, cons);
+
+    const int g = lane >> 2, q4 = lane & 3;  // head g; token / column pair q4
+    uint32_t qh[KC][2], ql[KC][2];            // A fragments of q (high, low): (head g, dims 2q4.., 2q4+8..)
+    float o[KC][4];                           // O^T: (dim 16i + g (+8), heads 2q4, 2q4 + 1)
+    float m_run = -INFINITY, l_run = 0.0f;    // head g (replicated over the quad)
+
+    for (int seq = 0; seq < ntile; ++seq) {
+        if (seq == 0 || cons.ti == 0) {  // a new context segment starts
+            const float *qb = p.q + (static_cast<size_t>(cons.r) * p.Hq + static_cast<size_t>(cons.h) * G + g) * D;
+#pragma unroll
+            for (int c = 0; c < KC; ++c) {
+                float2 x0 = make_float2(0.0f, 0.0f), x1 = x0;  // rows of heads past the group stay zero
+                if (g < G) {
+                    x0 = __ldg(reinterpret_cast<const float2 *>(qb + 16 * c + 2 * q4));
+                    x1 = __ldg(reinterpret_cast<const float2 *>(qb + 16 * c + 8 + 2 * q4));
+                }
+                split2<BF16>(x0.x * p.qscale, x0.y * p.qscale, qh[c][0], ql[c][0]);
+                split2<BF16>(x1.x * p.qscale, x1.y * p.qscale, qh[c][1], ql[c][1]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) o[c][e] = 0.0f;
+            }
+            m_run = -INFINITY;
+            l_run = 0.0f;
+        }
+
+        const int st = seq % NST;
+        const uint32_t par = (seq / NST) & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(kbar0 + st * 16, par))) {
+            if (lane == 0) report(p.status, KVP_ETIMEOUT, cons.r);
+            return;
+        }
+        const int nv = nvalid[st];
+        const uint32_t kt = ring + st * S::STAGE_BYTES, vt = kt + S::HALF_BYTES;
+        // ldmatrix row of this lane: matrix lane/8 covers tokens 8*(lane/16) ..
+        // and the 8-column chunk (lane/8) % 2 of each 16-column step
+        const int lrow = (lane & 7) + ((lane >> 4) << 3), lsub = (lane >> 3) & 1;
+        float sc[2][4];  // tokens 0-7 and 8-15
+        if (nv > 0) {
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sc[h2][e] = 0.0f;
+#pragma unroll
+            for (int c = 0; c < KC; ++c) {
+                uint32_t b[4];
+                ldsm_x4(tc_addr<D>(kt, lrow, 2 * c + lsub), b);
+                // b: (tokens 0-7: dims lo, hi), (tokens 8-15: dims lo, hi)
+                mma16816<BF16>(sc[0], qh[c][0], 0u, qh[c][1], 0u, b[0], b[1]);
+                mma16816<BF16>(sc[0], ql[c][0], 0u, ql[c][1], 0u, b[0], b[1]);
+                mma16816<BF16>(sc[1], qh[c][0], 0u, qh[c][1], 0u, b[2], b[3]);
+                mma16816<BF16>(sc[1], ql[c][0], 0u, ql[c][1], 0u, b[2], b[3]);
+            }
+        }
+        __syncwarp();  // K half is free
+        if (seq + NST < ntile) issue(seq + NST, 0, st);
+
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(kbar0 + st * 16 + 8, par))) {
+            if (lane == 0) report(p.status, KVP_ETIMEOUT, cons.r);
+            return;
+        }
+        if (nv > 0) {
+            // scores of head g at tokens 2q4, 2q4+1, 8+2q4, 9+2q4 (masked by select)
+            float x[4] = {sc[0][0], sc[0][1], sc[1][0], sc[1][1]};
+            const int t0 = 2 * q4;
+            if (t0 >= nv) x[0] = -INFINITY;
+            if (t0 + 1 >= nv) x[1] = -INFINITY;
+            if (t0 + 8 >= nv) x[2] = -INFINITY;
+            if (t0 + 9 >= nv) x[3] = -INFINITY;
+            float mt = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+            mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
+            mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
+            // lazy reference max (as in the CUDA-core kernel): it moves only
+            // when some score exceeds it by more than kLazy
+            if (__any_sync(0xffffffffu, mt > m_run + kLazy)) {
+                const float mn = fmaxf(m_run, mt);
+                const float alpha = (mn == m_run) ? 1.0f : ex2(m_run - mn);
+                m_run = mn;
+                l_run *= alpha;
+                const float aA = __shfl_sync(0xffffffffu, alpha, 8 * q4);      // head 2q4
+                const float aB = __shfl_sync(0xffffffffu, alpha, 8 * q4 + 4);  // head 2q4 + 1
+#pragma unroll
+                for (int c = 0; c < KC; ++c) {
+                    o[c][0] *= aA;
+                    o[c][1] *= aB;
+                    o[c][2] *= aA;
+                    o[c][3] *= aB;
+                }
+            }
+            float pr[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) pr[e] = ex2(x[e] - m_run);  // masked: exp2(-inf) = 0
+            uint32_t ph0, pl0, ph1, pl1;  // B fragments of P^T (tokens 2q4.., 8+2q4..; head g)
+            split2<BF16>(pr[0], pr[1], ph0, pl0);
+            split2<BF16>(pr[2], pr[3], ph1, pl1);
+            {
+                // the row sum adds exactly the weights the product uses (hi + lo)
+                const float2 h0 = unpack2<BF16>(ph0), l0 = unpack2<BF16>(pl0);
+                const float2 h1 = unpack2<BF16>(ph1), l1 = unpack2<BF16>(pl1);
+                l_run += ((h0.x + l0.x) + (h0.y + l0.y)) + ((h1.x + l1.x) + (h1.y + l1.y));
+            }
+            if (nv < TT) {
+                // V rows past the context may hold anything (never-written
+                // slots): zero them so 0 * V stays 0 in the product
+                const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+                for (int k = lane; k < (TT - nv) * (D / 8); k += 32) {
+                    const int row = nv + k / (D / 8), c8 = k % (D / 8);
+                    *reinterpret_cast<uint4 *>(smem + (tc_addr<D>(vt, row, c8) - smem_addr(smem))) = z;
+                }
+                __syncwarp();
+            }
+#pragma unroll
+            for (int c = 0; c < KC; ++c) {
+                uint32_t a[4];
+                // V^T rows (dims 16c ..), columns (tokens): transposed 8x8 loads
+                ldsm_x4_trans(tc_addr<D>(vt, (lane & 7) + ((lane >> 4) << 3), 2 * c + ((lane >> 3) & 1)), a);
+                mma16816<BF16>(o[c], a[0], a[1], a[2], a[3], ph0, ph1);
+                mma16816<BF16>(o[c], a[0], a[1], a[2], a[3], pl0, pl1);
+            }
+        }
+        __syncwarp();  // V half is free
+        if (seq + NST < ntile) issue(seq + NST, 1, st);
+
+        // ---- end of this warp's segment of the (r, h) context
+        if (cons.ti == cons.nt - 1 || seq == ntile - 1) {
+            const int r = cons.r, h = cons.h, nt = cons.nt;
+            float lh = l_run;
+            lh += __shfl_xor_sync(0xffffffffu, lh, 1);
+            lh += __shfl_xor_sync(0xffffffffu, lh, 2);
+            int w_first, w_last;
+            context_warps(s_cpref[r] + h * (nt + kCtxCost) + kCtxCost, nt, W, TC, w_first, w_last);
+            const bool whole = (w_first == w_last);
+            const float lA = __shfl_sync(0xffffffffu, lh, 8 * q4), lB = __shfl_sync(0xffffffffu, lh, 8 * q4 + 4);
+            float *dst;
+            float sA = 1.0f, sB = 1.0f;
+            if (whole) {
+                dst = p.out + (static_cast<size_t>(r) * p.Hq + static_cast<size_t>(h) * G) * D;
+                sA = lA > 0.0f ? 1.0f / lA : 0.0f;
+                sB = lB > 0.0f ? 1.0f / lB : 0.0f;
+            } else {
+                dst = part_slot<D, G>(p, w, r * Hkv + h);
+                if (q4 == 0 && g < G) {
+                    dst[G * D + 2 * g] = m_run;
+                    dst[G * D + 2 * g + 1] = lh;
+                }
+            }
+            if (2 * q4 < G) {  // this lane's heads 2q4, 2q4 + 1 are in the group
+#pragma unroll
+                for (int c = 0; c < KC; ++c) {
+                    const int d0 = 16 * c + g;
+                    dst[(2 * q4) * D + d0] = o[c][0] * sA;
+                    dst[(2 * q4 + 1) * D + d0] = o[c][1] * sB;
+                    dst[(2 * q4) * D + d0 + 8] = o[c][2] * sA;
+                    dst[(2 * q4 + 1) * D + d0 + 8] = o[c][3] * sB;
+                }
+            }
+        }
+        advance(cons);
+    }
+}
+
 // ------------------------------------------------------------ combine grid
 // Log-sum-exp merge for GridCombine group sizes: one warp per (context,
 // query head of the group). All segments' (max, sum) pairs come in one load
@@ -1072,8 +1496,17 @@ static int sm_count(int dev)
 template <int D, int G>
 static int warps_per_cta() { return Shape<D, G>::NW; }
 
-static int nw_for(int D, int G)
+// The tensor-core kernel serves groups of 4 and 8 query heads when a
+// 16-token tile lies inside one block (block size >= 16); the CUDA-core
+// kernel serves the rest (groups of 1 and 2, smaller blocks).
+static bool use_tc(const kvp_pool *pool, int G)
 {
+    return (G == 4 || G == 8) && pool->cfg.block_size >= TT && pool->cfg.head_dim % 64 == 0;
+}
+
+static int nw_for(int D, int G, bool tc)
+{
+    if (tc) return D <= 128 ? TcShape<128>::NW : TcShape<256>::NW;
 #define KVP_NW(d, g) \
     if (D == d && G == g) return warps_per_cta<d, g>();
     KVP_NW(64, 1) KVP_NW(64, 2) KVP_NW(64, 4) KVP_NW(64, 8)
@@ -1090,11 +1523,12 @@ struct Layout {
 
 static int plan(const kvp_pool *pool, int G, int Hkv, int B, int max_ctx, int split_req, Layout *L)
 {
+    const bool tc = use_tc(pool, G);
     if (split_req < 0 || split_req % TT)
         return set_error(KVP_EINVAL, "split_tokens %d must be 0 or a positive multiple of %d", split_req, TT);
     if (B < 0 || B > kMaxBatch) return set_error(KVP_EUNSUPPORTED, "B %d outside [0, %d]", B, kMaxBatch);
     if (max_ctx < 0) return set_error(KVP_EINVAL, "max_ctx_len must be >= 0");
-    const int nw = nw_for(pool->cfg.head_dim, G);
+    const int nw = nw_for(pool->cfg.head_dim, G, tc);
     if (!nw) return set_error(KVP_EUNSUPPORTED, "decode: head_dim %d with GQA group %d not built", pool->cfg.head_dim, G);
     const int sms = sm_count(pool->cfg.device);
     if (!sms) return set_error(KVP_ECUDA, "cannot query the SM count of device %d", pool->cfg.device);
@@ -1127,6 +1561,32 @@ static int launch(const Params &p, bool bf16, int blocks, cudaStream_t s)
                         "decode combine launch");
     }
     return rc;
+}
+
+// 8-head groups on the tensor-core kernel (block size >= 16: a tile is one
+// 16-row box inside one block), then the merge grid.
+template <int D, int G>
+static int launch_tc(const Params &p, const kvp_pool *pool, int layer, bool bf16, cudaStream_t s)
+{
+    const size_t smem = TcSmem<D>::total(p.B);
+    if (smem > 227 * 1024) return set_error(KVP_EUNSUPPORTED, "decode: %zu bytes of shared memory", smem);
+    CUtensorMap mk, mv;
+    int rc;
+    if ((rc = make_pool_tmap(&mk, pool->k_base + pool->layer_words * layer, pool, TT)) ||
+        (rc = make_pool_tmap(&mv, pool->v_base + pool->layer_words * layer, pool, TT)))
+        return rc;
+    auto kern = bf16 ? decode_tc_kernel<D, G, true> : decode_tc_kernel<D, G, false>;
+    if ((rc = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)),
+                         "decode smem attribute")))
+        return rc;
+    const int blocks = p.warps_total / TcShape<D>::NW;
+    if ((rc = check_cuda(launch_pdl(kern, dim3(blocks), dim3(TcShape<D>::NW * 32), smem, s, mk, mv, p), "decode launch")))
+        return rc;
+    const int tasks = p.B * p.Hkv * G;
+    const int cblocks = max(1, min((tasks + kCombineWarps - 1) / kCombineWarps, 4 * blocks));
+    const size_t csmem = align_up(sizeof(int) * (3 * static_cast<size_t>(p.B) + 2), 16);
+    return check_cuda(launch_pdl(combine_kernel<D, G>, dim3(cblocks), dim3(kCombineWarps * 32), csmem, s, p),
+                      "decode combine launch");
 }
 
 template <int D>
@@ -1190,8 +1650,21 @@ extern "C" int paged_decode_attention(kvp_pool *pool, int layer, const kvp_attn_
     const double scale = static_cast<double>(static_cast<float>(1.0 / sqrt(static_cast<double>(pool->cfg.head_dim))));
     p.qscale = static_cast<float>(scale * 1.4426950408889634);  // log2(e): softmax via exp2
     const bool bf16 = pool->cfg.kv_dtype == KVP_BF16;
-    const int blocks = L.warps_total / dec::nw_for(pool->cfg.head_dim, G);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dec::use_tc(pool, G)) {
+        const int D = pool->cfg.head_dim;
+        if (G == 8) {
+            if (D == 64) return dec::launch_tc<64, 8>(p, pool, layer, bf16, s);
+            if (D == 128) return dec::launch_tc<128, 8>(p, pool, layer, bf16, s);
+            if (D == 256) return dec::launch_tc<256, 8>(p, pool, layer, bf16, s);
+        } else {
+            if (D == 64) return dec::launch_tc<64, 4>(p, pool, layer, bf16, s);
+            if (D == 128) return dec::launch_tc<128, 4>(p, pool, layer, bf16, s);
+            if (D == 256) return dec::launch_tc<256, 4>(p, pool, layer, bf16, s);
+        }
+        return set_error(KVP_EUNSUPPORTED, "head_dim %d", D);
+    }
+    const int blocks = L.warps_total / dec::nw_for(pool->cfg.head_dim, G, false);
     switch (pool->cfg.head_dim) {
     case 64: return dec::launch_g<64>(p, bf16, blocks, G, s);
     case 128: return dec::launch_g<128>(p, bf16, blocks, G, s);

@@ -8,6 +8,8 @@
 
 #include <vector>
 
+#include <mutex>
+
 #include "common.cuh"
 
 namespace kvp {
@@ -234,3 +236,47 @@ int kvp_convert_bits(uint64_t start, int64_t count, int kv_dtype, uint16_t *out,
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------ tensor maps
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+}  // namespace
+
+int kvp::make_pool_tmap(CUtensorMap *map, const uint16_t *base, const kvp_pool *pool, int box_rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return set_error(KVP_ECUDA, "cuTensorMapEncodeTiled is unavailable");
+    const kvp_cache_config &c = pool->cfg;
+    if (box_rows < 1 || box_rows > c.block_size || box_rows > 256)
+        return set_error(KVP_EUNSUPPORTED, "tensor map box of %d rows over blocks of %d", box_rows, c.block_size);
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(c.head_dim), static_cast<cuuint64_t>(c.block_size),
+                          static_cast<cuuint64_t>(c.num_blocks) * c.num_kv_heads};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(c.head_dim) * 2,
+                             static_cast<cuuint64_t>(c.head_dim) * c.block_size * 2};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(map, c.kv_dtype == KVP_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                          3, const_cast<uint16_t *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return set_error(KVP_ECUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return KVP_OK;
+}

@@ -36,8 +36,6 @@
 
 #include <math.h>
 
-#include <mutex>
-
 #include "common.cuh"
 
 namespace kvp {
@@ -598,45 +596,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 }
 
 // ------------------------------------------------------------------- host
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_fn()
-{
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    });
-    return fn;
-}
-
-// Tensor map over one layer's pool viewed as [blocks*Hkv][bs][D] with a box of
-// 64 columns x bs rows x 1 tile and the 128-byte swizzle.
-static int make_map(CUtensorMap *map, const uint16_t *base, const kvp_pool *pool)
-{
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return set_error(KVP_ECUDA, "cuTensorMapEncodeTiled is unavailable");
-    const kvp_cache_config &c = pool->cfg;
-    cuuint64_t dims[3] = {static_cast<cuuint64_t>(c.head_dim), static_cast<cuuint64_t>(c.block_size),
-                          static_cast<cuuint64_t>(c.num_blocks) * c.num_kv_heads};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(c.head_dim) * 2,
-                             static_cast<cuuint64_t>(c.head_dim) * c.block_size * 2};
-    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(c.block_size), 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    const CUresult r = fn(map, c.kv_dtype == KVP_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                          3, const_cast<uint16_t *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return set_error(KVP_ECUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
-    return KVP_OK;
-}
-
 template <int G, bool BF16>
 static int launch(const CUtensorMap &mk, const CUtensorMap &mv, const Params &p, cudaStream_t s)
 {
@@ -687,7 +646,7 @@ extern "C" int paged_prefill_attention(kvp_pool *pool, int layer, const kvp_attn
     CUtensorMap mk, mv;
     const uint16_t *kp = pool->k_base + pool->layer_words * layer;
     const uint16_t *vp = pool->v_base + pool->layer_words * layer;
-    if ((rc = pre::make_map(&mk, kp, pool)) || (rc = pre::make_map(&mv, vp, pool))) return rc;
+    if ((rc = make_pool_tmap(&mk, kp, pool, bs)) || (rc = make_pool_tmap(&mv, vp, pool, bs))) return rc;
     pre::Params p;
     p.q = q, p.out = out, p.cu_q = cu_q, p.ctx = ctx_lens, p.bt = block_tables, p.status = pool->status;
     p.S = S, p.Hq = Hq, p.Hkv = Hkv, p.G = G, p.mbps = max_blocks_per_seq, p.bs = bs;
