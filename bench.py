@@ -75,6 +75,15 @@ def sources_sha(paths) -> str:
     return h.hexdigest()[:16]
 
 
+def decode_kernel_name(sp) -> str:
+    """The decode kernel the library picks for this shape (tensor-core tile
+    products for groups of 4 and 8 with blocks of at least 16 tokens)."""
+    G = sp.Hq // sp.Hkv
+    if G in (4, 8) and sp.bs >= 16 and sp.D % 64 == 0:
+        return "kvp::dec::decode_tc_kernel (+ merge grid)"
+    return "kvp::dec::decode_kernel"
+
+
 def ncu_traffic(workload: str):
     """DRAM bytes per decode launch from the committed ncu summary, or None
     when the kernel sources changed since that capture."""
@@ -424,7 +433,7 @@ def run_ours(args):
         "append_us_incl_gap": round((step_ms - dec_ms) * 1e3, 2),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "peak_kind": peak_kind, "kernel": "kvp::dec::decode_kernel"},
+                     "peak_kind": peak_kind, "kernel": decode_kernel_name(sp)},
         "clocks": clk,
         "e2e": {"value": round(total_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},

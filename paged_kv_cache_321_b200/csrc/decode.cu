@@ -410,6 +410,7 @@ __device__ __noinline__ void combine(const Params &p, int rh, int w_first, int w
     }
 }
 
+constexpr bool kGridMerge4 = false;
 // With 8 query heads per kv head the streaming loop already needs every
 // register a thread can have; any merge code inside it costs spills there.
 // Those contexts are merged by a separate grid instead (combine_kernel),
@@ -417,7 +418,7 @@ __device__ __noinline__ void combine(const Params &p, int rh, int w_first, int w
 // G warps rather than run by one.
 template <int G>
 struct GridCombine {
-    static constexpr bool value = G >= 8;
+    static constexpr bool value = G >= 8 || kGridMerge4;
 };
 
 // GPU-scope fence with acquire-release semantics. Before a count: this
@@ -958,8 +959,8 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
 // deliver the tile (8 heads: twice as many), so this variant does both
 // contractions of a tile with warp-level mma.sync (m16n8k16, 16-bit inputs,
 // fp32 accumulation); the rest of the design is unchanged (persistent,
-// stream-K in cost space, per-warp rings), the split partials go to the
-// merge grid:
+// stream-K in cost space, per-warp rings, split partials merged by the last
+// warp of a context for groups of 4 and by the merge grid for groups of 8):
 //  * S = Q K^T: A = the group's query heads (rows past the group and rows
 //    8..15 zero), B = the K tile as loaded; q is split into a 16-bit high
 //    part and the 16-bit rounding of the remainder, both multiplied, so the
@@ -1215,6 +1216,8 @@ __global__ void __launch_bounds__(TcShape<D>::NW * 32, 1)
     uint32_t qh[KC][2], ql[KC][2];            // A fragments of q (high, low): (head g, dims 2q4.., 2q4+8..)
     float o[KC][4];                           // O^T: (dim 16i + g (+8), heads 2q4, 2q4 + 1)
     float m_run = -INFINITY, l_run = 0.0f;    // head g (replicated over the quad)
+    // split segments to count in (groups merged in the kernel, as in decode_kernel)
+    int npub = 0, rh0 = 0, wf0 = 0, wl0 = 0, rh1 = 0, wf1 = 0, wl1 = 0, old0 = -1;
 
     for (int seq = 0; seq < ntile; ++seq) {
         if (seq == 0 || cons.ti == 0) {  // a new context segment starts
@@ -1365,8 +1368,52 @@ __global__ void __launch_bounds__(TcShape<D>::NW * 32, 1)
                     dst[(2 * q4 + 1) * D + d0 + 8] = o[c][3] * sB;
                 }
             }
+            if constexpr (!GridCombine<G>::value) {
+                if (!whole) {
+                    if (npub++ == 0) {
+                        rh0 = r * Hkv + h, wf0 = w_first, wl0 = w_last;
+                        if (seq != ntile - 1) {  // counted in now, the reply looked at later
+                            __syncwarp();
+                            if (lane == 0) {
+                                fence_acq_rel_gpu();
+                                old0 = atomic_add_relaxed(&p.counters[rh0], 1);
+                            }
+                        }
+                    } else {
+                        rh1 = r * Hkv + h, wf1 = w_first, wl1 = w_last;
+                    }
+                }
+            }
         }
         advance(cons);
+    }
+
+    if constexpr (!GridCombine<G>::value) {
+        // count the range's split segments in; the warp that completes a
+        // count merges that context and resets its counter
+        if (npub > 0) {
+            __syncwarp();
+            int last0 = 0, last1 = 0;
+            if (lane == 0) {
+                fence_acq_rel_gpu();
+                if (old0 < 0) old0 = atomic_add_relaxed(&p.counters[rh0], 1);
+                const int old1 = npub > 1 ? atomic_add_relaxed(&p.counters[rh1], 1) : -1;
+                last0 = old0 == wl0 - wf0;
+                last1 = npub > 1 && old1 == wl1 - wf1;
+                if (last0 || last1) fence_acq_rel_gpu();
+            }
+            last0 = __shfl_sync(0xffffffffu, last0, 0);
+            last1 = __shfl_sync(0xffffffffu, last1, 0);
+            __syncwarp();
+            if (last0) {
+                combine<D, G>(p, rh0, wf0, wl0, lane, p.out + static_cast<size_t>(rh0) * G * D);
+                if (lane == 0) p.counters[rh0] = 0;
+            }
+            if (last1) {
+                combine<D, G>(p, rh1, wf1, wl1, lane, p.out + static_cast<size_t>(rh1) * G * D);
+                if (lane == 0) p.counters[rh1] = 0;
+            }
+        }
     }
 }
 
@@ -1582,6 +1629,7 @@ static int launch_tc(const Params &p, const kvp_pool *pool, int layer, bool bf16
     const int blocks = p.warps_total / TcShape<D>::NW;
     if ((rc = check_cuda(launch_pdl(kern, dim3(blocks), dim3(TcShape<D>::NW * 32), smem, s, mk, mv, p), "decode launch")))
         return rc;
+    if constexpr (!GridCombine<G>::value) return KVP_OK;  // merged inside the kernel
     const int tasks = p.B * p.Hkv * G;
     const int cblocks = max(1, min((tasks + kCombineWarps - 1) / kCombineWarps, 4 * blocks));
     const size_t csmem = align_up(sizeof(int) * (3 * static_cast<size_t>(p.B) + 2), 16);
