@@ -410,7 +410,6 @@ __device__ __noinline__ void combine(const Params &p, int rh, int w_first, int w
     }
 }
 
-constexpr bool kGridMerge4 = false;
 // With 8 query heads per kv head the streaming loop already needs every
 // register a thread can have; any merge code inside it costs spills there.
 // Those contexts are merged by a separate grid instead (combine_kernel),
@@ -418,7 +417,7 @@ constexpr bool kGridMerge4 = false;
 // G warps rather than run by one.
 template <int G>
 struct GridCombine {
-    static constexpr bool value = G >= 8 || kGridMerge4;
+    static constexpr bool value = G >= 8;
 };
 
 // GPU-scope fence with acquire-release semantics. Before a count: this
