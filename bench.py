@@ -255,9 +255,22 @@ def run_ours(args):
     rope = torch.empty(wl.max_seq_len * sp.D, dtype=torch.float32, device=dev)
     K.rope_table_fill(attn, wl.max_seq_len, rope)
     g = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(dev)
-    q, k, v = g(wl.q), g(wl.k), g(wl.v)
+    # the step's per-step inputs live in one device buffer (256-byte aligned
+    # views), so the end-to-end leg below moves them with one host->device copy
+    step_inputs = [np.ascontiguousarray(a) for a in (wl.q, wl.k, wl.v, wl.tok_req, wl.positions, wl.block_tables,
+                                                      wl.ctx)]
+    offs, nbytes = [], 0
+    for a in step_inputs:
+        offs.append(nbytes)
+        nbytes += (a.nbytes + 255) // 256 * 256
+    h_pack = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    for a, o in zip(step_inputs, offs):
+        h_pack[o:o + a.nbytes].copy_(torch.from_numpy(a.view(np.uint8).reshape(-1)))
+    d_pack = h_pack.to(dev)
+    views = [d_pack[o:o + a.nbytes].view(torch.from_numpy(a[:0]).dtype).view(a.shape)
+             for a, o in zip(step_inputs, offs)]
+    q, k, v, tok_req, positions, bt, ctx = views
     qn, kn = g(wl.q_norm_w), g(wl.k_norm_w)
-    tok_req, positions, bt, ctx = g(wl.tok_req), g(wl.positions), g(wl.block_tables), g(wl.ctx)
     dseq, pseq = wl.decode_seqs, wl.prefill_seqs
     T = wl.T
     q_out = torch.empty((T, sp.Hq * sp.D), dtype=torch.float32, device=dev)
@@ -331,7 +344,7 @@ def run_ours(args):
         if dist is not None:
             dist.barrier()
 
-    # ---- device-resident timing: K steps, events around every decode and prefill launch
+    # ---- device-resident timing
     def step(i=None):
         append()
         gather_q()
@@ -354,13 +367,23 @@ def run_ours(args):
     evp = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     clocks = ClockSampler(dev.index)
     clocks.start()
+    # (1) K steps back to back, events only around the whole run: the kernels
+    # of a step are launched with programmatic dependencies, and an event
+    # recorded between two of them would stop the next one's launch from
+    # overlapping the previous one, so per-kernel events stay out of this run
     barrier()
     torch.cuda.synchronize()
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
     for i in range(args.steps):
-        step(i)
+        step()
     t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    # (2) the same K steps with events around every decode and prefill launch:
+    # the kernels' own durations for the roofline
+    for i in range(args.steps):
+        step(i)
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
@@ -372,18 +395,15 @@ def run_ours(args):
 
     # ---- end to end through the C ABI with host buffers: H2D of the step's
     # inputs from pinned memory, the step, D2H of the attention output
-    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
-    h_in = [pin(wl.q), pin(wl.k), pin(wl.v), pin(wl.tok_req), pin(wl.positions), pin(wl.block_tables),
-            pin(wl.ctx)]
-    d_in = [q, k, v, tok_req, positions, bt, ctx]
+    # (q, k, v, token -> sequence, positions, block tables and context lengths
+    # in one pinned buffer, one copy; the decode output back)
     h_out = torch.empty(out.shape, dtype=torch.float32).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in h_in)
+    h2d = sum(a.nbytes for a in step_inputs)
     d2h = h_out.numel() * h_out.element_size()
     e2e_steps = max(1, min(args.steps, 500))
 
     def e2e_step():
-        for h, d in zip(h_in, d_in):
-            d.copy_(h, non_blocking=True)
+        d_pack.copy_(h_pack, non_blocking=True)
         step()
         h_out.copy_(out, non_blocking=True)
 
