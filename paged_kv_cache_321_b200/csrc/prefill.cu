@@ -483,13 +483,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_SFREE + b));
-            // causal mask and row max (this half, then both)
+            // causal mask (skipped when all 64 keys are visible to every row
+            // of the warp, as for all but the diagonal tiles) and row max
             const int key0 = j * BN + col0;
             float mx = -INFINITY;
+            if (__all_sync(0xffffffffu, key0 + 63 <= pos)) {
 #pragma unroll
-            for (int i = 0; i < 64; ++i) {
-                if (key0 + i > pos) sv[i] = -INFINITY;
-                mx = fmaxf(mx, sv[i]);
+                for (int i = 0; i < 64; ++i) mx = fmaxf(mx, sv[i]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 64; ++i) {
+                    if (key0 + i > pos) sv[i] = -INFINITY;
+                    mx = fmaxf(mx, sv[i]);
+                }
             }
             float mo;
             if (!exchange(j, mx, mo)) {
@@ -534,8 +540,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float x0 = sv[c * 8 + 2 * e], x1 = sv[c * 8 + 2 * e + 1];
-                    const float p0 = (x0 == -INFINITY) ? 0.0f : ex2(x0 - m_ref);
-                    const float p1 = (x1 == -INFINITY) ? 0.0f : ex2(x1 - m_ref);
+                    // a masked score gives exp2(-inf) = 0; m_ref is finite from
+                    // the first tile on in every row that has a query (key 0 is
+                    // visible to all), rows past the chunk are never stored
+                    const float p0 = ex2(x0 - m_ref);
+                    const float p1 = ex2(x1 - m_ref);
                     w[e] = pack2<BF16>(p0, p1);
                     const float2 back = unpack<BF16>(w[e]);
                     l += back.x + back.y;
