@@ -112,7 +112,7 @@ struct Smem {
     static constexpr size_t bars = static_cast<size_t>(S::NW) * NST * S::STAGE_BYTES;
     static constexpr size_t masks = bars + S::NW * NST * 2 * 8;
     static constexpr size_t pbuf = align_up(masks + S::NW * NST * 4, 16);
-    static constexpr size_t tiles = pbuf + S::NW * TT * G * 8;  // [B] tiles per sequence
+    static constexpr size_t tiles = pbuf + S::NW * TT * G * 8;  // [B] context lengths
     __host__ __device__ static size_t pref(int B) { return align_up(tiles + 4 * static_cast<size_t>(B), 16); }  // [B + 1]
     __host__ __device__ static size_t cpref(int B) { return align_up(pref(B) + 4 * static_cast<size_t>(B + 1), 16); }  // [B + 1]
     __host__ __device__ static size_t total(int B) { return align_up(cpref(B) + 4 * static_cast<size_t>(B + 1), 128); }
@@ -211,16 +211,20 @@ __device__ __forceinline__ bool ctx_ok(const Params &p, int c)
 // kCtxCost empty units, so such a warp gets about one tile less.
 constexpr int kCtxCost = 1;
 
+// The kernels keep each sequence's context length in shared memory (-1 for
+// one the kernel refuses), and derive its number of tiles from it.
+__device__ __forceinline__ int tiles_of(int ctx) { return ctx > 0 ? (ctx + TT - 1) / TT : 0; }
+
 // Exclusive prefixes over the B sequences, by one warp: s_pref[i] of the
-// tiles (s_tiles * Hkv), s_cpref[i] of the cost units (Hkv * (tiles +
+// tiles (tiles_of(s_ctx) * Hkv), s_cpref[i] of the cost units (Hkv * (tiles +
 // kCtxCost) for a sequence with tiles). s_pref[B] is the number of tiles,
 // s_cpref[B] the length of the cost space.
-__device__ __forceinline__ void tile_prefix(const int *s_tiles, int *s_pref, int *s_cpref, int B, int Hkv, int lane)
+__device__ __forceinline__ void tile_prefix(const int *s_ctx, int *s_pref, int *s_cpref, int B, int Hkv, int lane)
 {
     int run = 0, crun = 0;
     for (int base = 0; base < B; base += 32) {
         const int i = base + lane;
-        const int nt = i < B ? s_tiles[i] : 0;
+        const int nt = i < B ? tiles_of(s_ctx[i]) : 0;
         const int v = nt * Hkv, cv = nt > 0 ? (nt + kCtxCost) * Hkv : 0;
         int x = v, cx = cv;
 #pragma unroll
@@ -245,7 +249,7 @@ __device__ __forceinline__ int active_warps(const Params &p, int total)
 // Warp w owns the cost units [floor(w*TC/W), floor((w+1)*TC/W)). The first
 // tile whose cost position is at least U (the tiles of context (r, h) sit at
 // cost positions s_cpref[r] + h*(nt + kCtxCost) + kCtxCost + i).
-__device__ __forceinline__ int cost_to_tile(int64_t U, const int *s_tiles, const int *s_pref, const int *s_cpref,
+__device__ __forceinline__ int cost_to_tile(int64_t U, const int *s_ctx, const int *s_pref, const int *s_cpref,
                                             int B)
 {
     if (U >= s_cpref[B]) return s_pref[B];
@@ -255,7 +259,7 @@ __device__ __forceinline__ int cost_to_tile(int64_t U, const int *s_tiles, const
         if (s_cpref[mid] <= U) lo = mid;
         else hi = mid;
     }
-    const int nt = s_tiles[lo], span = nt + kCtxCost;
+    const int nt = tiles_of(s_ctx[lo]), span = nt + kCtxCost;
     const int local = static_cast<int>(U - s_cpref[lo]);
     const int h = local / span, off = local - h * span;
     return s_pref[lo] + h * nt + max(0, off - kCtxCost);
@@ -446,7 +450,7 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + M::bars);
     uint32_t *masks = reinterpret_cast<uint32_t *>(smem + M::masks);
     float2 *pbuf = reinterpret_cast<float2 *>(smem + M::pbuf);
-    int *s_tiles = reinterpret_cast<int *>(smem + M::tiles);
+    int *s_ctx = reinterpret_cast<int *>(smem + M::tiles);  // context lengths
     int *s_pref = reinterpret_cast<int *>(smem + M::pref(p.B));
     int *s_cpref = reinterpret_cast<int *>(smem + M::cpref(p.B));
 
@@ -470,7 +474,7 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
     for (int i = tid; i < B; i += NW * 32) {
         const int c = p.ctx[i];
         const bool ok = ctx_ok(p, c);
-        s_tiles[i] = ok ? (c + TT - 1) / TT : 0;
+        s_ctx[i] = ok ? c : -1;
         if (blockIdx.x == 0 && (!ok || c == 0)) {
             if (!ok) report(p.status, KVP_ERANGE, i);
             float4 *o = reinterpret_cast<float4 *>(p.out + static_cast<size_t>(i) * p.Hq * D);
@@ -478,7 +482,7 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
         }
     }
     __syncthreads();
-    if (warp == 0) tile_prefix(s_tiles, s_pref, s_cpref, B, Hkv, lane);
+    if (warp == 0) tile_prefix(s_ctx, s_pref, s_cpref, B, Hkv, lane);
     __syncthreads();
 
     grid_launch_dependents();  // the next grid may be placed (it waits for this one)
@@ -488,8 +492,8 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
     const int W = active_warps(p, total);
     const int w = blockIdx.x * NW + warp;
     if (w >= W) return;
-    const int t_begin = cost_to_tile(static_cast<int64_t>(w) * TC / W, s_tiles, s_pref, s_cpref, B);
-    const int t_end = cost_to_tile(static_cast<int64_t>(w + 1) * TC / W, s_tiles, s_pref, s_cpref, B);
+    const int t_begin = cost_to_tile(static_cast<int64_t>(w) * TC / W, s_ctx, s_pref, s_cpref, B);
+    const int t_end = cost_to_tile(static_cast<int64_t>(w + 1) * TC / W, s_ctx, s_pref, s_cpref, B);
     if (t_begin >= t_end) return;  // no CTA-wide barrier follows
 
     // barriers: [warp][stage][K, V] "tile half landed"
@@ -507,7 +511,7 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
         }
         c.t = t;
         c.r = lo;
-        c.nt = s_tiles[lo];
+        c.nt = tiles_of(s_ctx[lo]);
         const int local = t - s_pref[lo];
         c.h = local / c.nt;
         c.ti = local - c.h * c.nt;
@@ -520,8 +524,8 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
                 c.h = 0;
                 do {
                     ++c.r;
-                } while (c.r < B && s_tiles[c.r] == 0);
-                if (c.r < B) c.nt = s_tiles[c.r];
+                } while (c.r < B && tiles_of(s_ctx[c.r]) == 0);
+                if (c.r < B) c.nt = tiles_of(s_ctx[c.r]);
             }
         }
     };
@@ -550,7 +554,7 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
             locate(t_begin + i, c);
             // a segment starts here: its queries are wanted when this tile is
             if (c.ti == 0 || i == 0) d_q = c.r * p.Hq + c.h * G;
-            const int ctx = p.ctx[c.r];
+            const int ctx = s_ctx[c.r];
             const int tb = c.ti * TT;
             const int blk = p.bt[static_cast<size_t>(c.r) * p.mbps + tb / p.bs];
             if (blk >= 0 && blk < p.num_blocks) {
@@ -566,7 +570,7 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
     auto issue_small = [&](int i, int half, int st) {
         Cursor c;
         locate(t_begin + i, c);
-        const int ctx = p.ctx[c.r];
+        const int ctx = s_ctx[c.r];
         const int tb = c.ti * TT;
         const int32_t *btr = p.bt + static_cast<size_t>(c.r) * p.mbps;
         const uint32_t bar = kbar0 + (st * 2 + half) * 8;
@@ -1072,7 +1076,7 @@ __global__ void __launch_bounds__(TcShape<D>::NW * 32, 1)
     unsigned char *smem = tc_smem;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + M::bars);
     int *nvalid_all = reinterpret_cast<int *>(smem + M::masks);
-    int *s_tiles = reinterpret_cast<int *>(smem + M::tiles);
+    int *s_ctx = reinterpret_cast<int *>(smem + M::tiles);  // context lengths
     int *s_pref = reinterpret_cast<int *>(smem + M::pref(p.B));
     int *s_cpref = reinterpret_cast<int *>(smem + M::cpref(p.B));
 
@@ -1093,7 +1097,7 @@ __global__ void __launch_bounds__(TcShape<D>::NW * 32, 1)
     for (int i = tid; i < B; i += NW * 32) {
         const int c = p.ctx[i];
         const bool ok = ctx_ok(p, c);
-        s_tiles[i] = ok ? (c + TT - 1) / TT : 0;
+        s_ctx[i] = ok ? c : -1;
         if (blockIdx.x == 0 && (!ok || c == 0)) {
             if (!ok) report(p.status, KVP_ERANGE, i);
             float4 *o = reinterpret_cast<float4 *>(p.out + static_cast<size_t>(i) * p.Hq * D);
@@ -1101,7 +1105,7 @@ __global__ void __launch_bounds__(TcShape<D>::NW * 32, 1)
         }
     }
     __syncthreads();
-    if (warp == 0) tile_prefix(s_tiles, s_pref, s_cpref, B, Hkv, lane);
+    if (warp == 0) tile_prefix(s_ctx, s_pref, s_cpref, B, Hkv, lane);
     __syncthreads();
     grid_launch_dependents();
 
@@ -1109,8 +1113,8 @@ __global__ void __launch_bounds__(TcShape<D>::NW * 32, 1)
     const int W = active_warps(p, total);
     const int w = blockIdx.x * NW + warp;
     if (w >= W) return;
-    const int t_begin = cost_to_tile(static_cast<int64_t>(w) * TC / W, s_tiles, s_pref, s_cpref, B);
-    const int t_end = cost_to_tile(static_cast<int64_t>(w + 1) * TC / W, s_tiles, s_pref, s_cpref, B);
+    const int t_begin = cost_to_tile(static_cast<int64_t>(w) * TC / W, s_ctx, s_pref, s_cpref, B);
+    const int t_end = cost_to_tile(static_cast<int64_t>(w + 1) * TC / W, s_ctx, s_pref, s_cpref, B);
     if (t_begin >= t_end) return;  // no CTA-wide barrier follows
 
     const uint32_t kbar0 = smem_addr(&bars[warp * NST * 2]);
@@ -1127,7 +1131,7 @@ __global__ void __launch_bounds__(TcShape<D>::NW * 32, 1)
         }
         c.t = t;
         c.r = lo;
-        c.nt = s_tiles[lo];
+        c.nt = tiles_of(s_ctx[lo]);
         const int local = t - s_pref[lo];
         c.h = local / c.nt;
         c.ti = local - c.h * c.nt;
@@ -1140,8 +1144,8 @@ __global__ void __launch_bounds__(TcShape<D>::NW * 32, 1)
                 c.h = 0;
                 do {
                     ++c.r;
-                } while (c.r < B && s_tiles[c.r] == 0);
-                if (c.r < B) c.nt = s_tiles[c.r];
+                } while (c.r < B && tiles_of(s_ctx[c.r]) == 0);
+                if (c.r < B) c.nt = tiles_of(s_ctx[c.r]);
             }
         }
     };
@@ -1164,7 +1168,7 @@ __global__ void __launch_bounds__(TcShape<D>::NW * 32, 1)
             Cursor c;
             locate(t_begin + i, c);
             if (c.ti == 0 || i == 0) d_q = c.r * p.Hq + c.h * G;
-            const int ctx = p.ctx[c.r];
+            const int ctx = s_ctx[c.r];
             const int tb = c.ti * TT;
             const int blk = p.bt[static_cast<size_t>(c.r) * p.mbps + tb / p.bs];
             if (blk >= 0 && blk < p.num_blocks) {
@@ -1431,7 +1435,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const Param
     constexpr int SL = slot_floats(G, D);
     constexpr int DL = D / 32;  // output dims per lane: 2, 4 or 8
     extern __shared__ __align__(16) int csm[];
-    int *s_tiles = csm;
+    int *s_ctx = csm;
     int *s_pref = csm + p.B;
     int *s_cpref = s_pref + p.B + 1;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1441,10 +1445,10 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const Param
     // waited for its predecessor), so they may be read before it finishes.
     for (int i = tid; i < B; i += kCombineWarps * 32) {
         const int c = p.ctx[i];
-        s_tiles[i] = ctx_ok(p, c) ? (c + TT - 1) / TT : 0;
+        s_ctx[i] = ctx_ok(p, c) ? c : -1;
     }
     __syncthreads();
-    if (warp == 0) tile_prefix(s_tiles, s_pref, s_cpref, B, Hkv, lane);
+    if (warp == 0) tile_prefix(s_ctx, s_pref, s_cpref, B, Hkv, lane);
     __syncthreads();
     const int total = s_pref[B], TC = s_cpref[B];
     const int W = active_warps(p, total);
@@ -1456,7 +1460,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const Param
     for (int task = blockIdx.x * kCombineWarps + warp; task < ntask; task += gridDim.x * kCombineWarps) {
         const int g = task % G, rh = task / G;
         const int r = rh / Hkv, h = rh - r * Hkv;
-        const int nt = s_tiles[r];
+        const int nt = tiles_of(s_ctx[r]);
         if (nt == 0) continue;
         int w_first, w_last;
         context_warps(s_cpref[r] + h * (nt + kCtxCost) + kCtxCost, nt, W, TC, w_first, w_last);
