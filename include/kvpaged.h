@@ -280,6 +280,82 @@ int kvp_convert_bits(uint64_t start, int64_t count, int kv_dtype, uint16_t *out,
 /* Library version: major * 10000 + minor * 100 + patch. */
 int kvp_version(void);
 
+/* -------------------------------------------- host block manager (prefix cache)
+ *
+ * Host-only bookkeeping that turns requests' token streams into block ids:
+ * per-layer block allocation with rollback and prefix caching, after
+ * PagedKVCache (ensureCapacityLocked, AppendToken, AllocateForTokens, Commit,
+ * Free, LayerBlockIDs) in makarna/pkg/kvcache/paged_cache.go. The page does
+ * not show the BlockPool it calls; the reading taken:
+ *   - a block is free, held (one reference per sequence holding it: its owner
+ *     and every borrower), or cached and unheld (findable by its hash until
+ *     evicted);
+ *   - allocation takes free blocks first, then evicts the least recently
+ *     released cached blocks; it takes all it needs or nothing;
+ *   - a block whose last reference goes is cached if it has a hash, else freed;
+ *   - a full block's hash is 64-bit FNV-1a over (a parent flag, the parent
+ *     block's hash, the block's token ids as little-endian int32); a prompt's
+ *     cached prefix is the longest run of its chained hashes present in every
+ *     layer, and its blocks are borrowed (never to be written: kv_append must
+ *     not target them);
+ *   - Commit publishes the blocks it completes, the first block per hash wins.
+ * All calls are host calls (no CUDA); calls on one kvp_blocks are serialised
+ * by its mutex. Errors: KVP_EINVAL (bad argument), KVP_ERANGE (not enough
+ * free blocks: nothing is taken), KVP_EOVERFLOW (beyond max_seq_len). The
+ * block ids index the pool of kv_pool_create (num_blocks must match). */
+typedef struct kvp_blocks kvp_blocks;
+typedef struct kvp_seq kvp_seq;
+
+/* A manager of num_blocks blocks per layer. max_seq_len = 0: no limit. */
+int kvp_blocks_create(int num_layers, int num_blocks, int block_size, int max_seq_len, kvp_blocks **out);
+int kvp_blocks_destroy(kvp_blocks *blocks); /* sequences must be destroyed first */
+
+/* Free, cached-unheld and held block counts of one layer (any may be NULL). */
+int kvp_blocks_count(kvp_blocks *blocks, int layer, int *free_blocks, int *cached_blocks, int *held_blocks);
+
+/* References held on one block (>= 0), or an error code. */
+int kvp_blocks_refs(kvp_blocks *blocks, int layer, int block);
+
+/* The chained hash of one full block of n token ids (parent NULL for the
+ * first block of a sequence). */
+uint64_t kvp_block_hash(const int32_t *tokens, int n, const uint64_t *parent);
+
+/* A sequence (request) with no blocks; destroy releases its blocks. */
+int kvp_seq_create(kvp_blocks *blocks, kvp_seq **out);
+int kvp_seq_destroy(kvp_seq *seq);
+
+/* Releases every block the sequence holds and forgets its tokens (Free). */
+int kvp_seq_free(kvp_seq *seq);
+
+/* A prompt of n tokens (AllocateForTokens): releases what the sequence held,
+ * borrows the cached prefix, allocates blocks for the rest of the prompt's
+ * full blocks in every layer (all or nothing), and sets *computed to the
+ * tokens whose K/V are already cached -- never all n: the last prompt token
+ * is always computed. */
+int kvp_seq_allocate_for_tokens(kvp_seq *seq, const int32_t *tokens, int n, int *computed);
+
+/* One more token (AppendToken): when it completes a block, the block is
+ * allocated if needed and hashed. */
+int kvp_seq_append_token(kvp_seq *seq, int32_t token);
+
+/* Blocks for num_tokens positions in every layer (ensureCapacityLocked; new
+ * blocks are owned; on failure nothing is kept from this call). */
+int kvp_seq_reserve(kvp_seq *seq, int num_tokens);
+
+/* new_tokens more tokens are computed (Commit): completed blocks with hashes
+ * are published to the prefix cache. */
+int kvp_seq_commit(kvp_seq *seq, int new_tokens);
+
+/* Computed tokens, and blocks held per layer. */
+int kvp_seq_len(const kvp_seq *seq);
+int kvp_seq_num_blocks(const kvp_seq *seq);
+
+/* One layer's block-table row (LayerBlockIDs): out[0..max_blocks) gets the
+ * block ids and -1 past them; owned (may be NULL) gets 1 for owned, 0 for
+ * borrowed. Returns the number of blocks, or KVP_ERANGE when max_blocks is
+ * too small. */
+int kvp_seq_block_table(const kvp_seq *seq, int layer, int32_t *out, int max_blocks, uint8_t *owned);
+
 #ifdef __cplusplus
 }
 #endif

@@ -15,10 +15,13 @@ from ._native import (  # noqa: F401
     KVP_F16,
     KVP_OK,
     AttnConfig,
+    Blocks,
     CacheConfig,
     KvpError,
     Pool,
+    Sequence,
     attn_config,
+    block_hash,
     convert_bits,
     convert_f32,
     decode_workspace_size,

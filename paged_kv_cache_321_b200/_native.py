@@ -30,6 +30,9 @@ EXPORTS = (
     "kvp_rope_table_bytes", "kvp_rope_table_fill", "kv_append", "paged_decode_workspace_size",
     "paged_decode_attention", "paged_decode_attention_noalloc", "paged_prefill_workspace_size", "paged_prefill_attention", "kvp_convert_f32",
     "kvp_convert_bits", "kvp_version",
+    "kvp_blocks_create", "kvp_blocks_destroy", "kvp_blocks_count", "kvp_blocks_refs", "kvp_block_hash",
+    "kvp_seq_create", "kvp_seq_destroy", "kvp_seq_free", "kvp_seq_allocate_for_tokens", "kvp_seq_append_token",
+    "kvp_seq_reserve", "kvp_seq_commit", "kvp_seq_len", "kvp_seq_num_blocks", "kvp_seq_block_table",
 )
 
 
@@ -79,6 +82,21 @@ def lib() -> C.CDLL:
             "kvp_convert_f32": (i32, [P, P, i64, i32, P]),
             "kvp_convert_bits": (i32, [u64, i64, i32, P, P]),
             "kvp_version": (i32, []),
+            "kvp_blocks_create": (i32, [i32, i32, i32, i32, C.POINTER(P)]),
+            "kvp_blocks_destroy": (i32, [P]),
+            "kvp_blocks_count": (i32, [P, i32, C.POINTER(i32), C.POINTER(i32), C.POINTER(i32)]),
+            "kvp_blocks_refs": (i32, [P, i32, i32]),
+            "kvp_block_hash": (u64, [P, i32, C.POINTER(u64)]),
+            "kvp_seq_create": (i32, [P, C.POINTER(P)]),
+            "kvp_seq_destroy": (i32, [P]),
+            "kvp_seq_free": (i32, [P]),
+            "kvp_seq_allocate_for_tokens": (i32, [P, P, i32, C.POINTER(i32)]),
+            "kvp_seq_append_token": (i32, [P, C.c_int32]),
+            "kvp_seq_reserve": (i32, [P, i32]),
+            "kvp_seq_commit": (i32, [P, i32]),
+            "kvp_seq_len": (i32, [P]),
+            "kvp_seq_num_blocks": (i32, [P]),
+            "kvp_seq_block_table": (i32, [P, i32, P, i32, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -226,3 +244,90 @@ def convert_f32(x: torch.Tensor, out: torch.Tensor, kv_dtype: str, stream=None):
 
 def convert_bits(start: int, count: int, kv_dtype: str, out: torch.Tensor, stream=None):
     _check(lib().kvp_convert_bits(start, count, DTYPE_CODES[kv_dtype], _ptr(out), _stream(stream)))
+
+
+# ------------------------------------------------------- host block manager
+class Blocks:
+    """Per-layer block allocator with a prefix cache (host only; see
+    include/kvpaged.h). Block ids index a Pool of the same num_blocks."""
+
+    def __init__(self, num_layers: int, num_blocks: int, block_size: int, max_seq_len: int = 0):
+        self.num_layers, self.num_blocks, self.block_size = num_layers, num_blocks, block_size
+        h = C.c_void_p()
+        _check(lib().kvp_blocks_create(num_layers, num_blocks, block_size, max_seq_len, C.byref(h)))
+        self.handle = h
+
+    def counts(self, layer: int = 0):
+        """(free, cached and unheld, held) blocks of a layer."""
+        f, c, h = C.c_int(), C.c_int(), C.c_int()
+        _check(lib().kvp_blocks_count(self.handle, layer, C.byref(f), C.byref(c), C.byref(h)))
+        return f.value, c.value, h.value
+
+    def refs(self, layer: int, block: int) -> int:
+        rc = lib().kvp_blocks_refs(self.handle, layer, block)
+        if rc < 0:
+            _check(rc)
+        return rc
+
+    def sequence(self) -> "Sequence":
+        return Sequence(self)
+
+    def close(self):
+        if self.handle:
+            lib().kvp_blocks_destroy(self.handle)
+            self.handle = None
+
+
+def block_hash(tokens, parent: Optional[int] = None) -> int:
+    arr = (C.c_int32 * len(tokens))(*[int(t) for t in tokens])
+    par = C.c_uint64(parent) if parent is not None else None
+    return lib().kvp_block_hash(arr, len(tokens), C.byref(par) if par is not None else None)
+
+
+class Sequence:
+    """One request's blocks in every layer (PagedKVCache's per-request state)."""
+
+    def __init__(self, blocks: Blocks):
+        self.blocks = blocks
+        h = C.c_void_p()
+        _check(lib().kvp_seq_create(blocks.handle, C.byref(h)))
+        self.handle = h
+
+    def allocate_for_tokens(self, tokens) -> int:
+        arr = (C.c_int32 * len(tokens))(*[int(t) for t in tokens])
+        computed = C.c_int()
+        _check(lib().kvp_seq_allocate_for_tokens(self.handle, arr, len(tokens), C.byref(computed)))
+        return computed.value
+
+    def append_token(self, token: int):
+        _check(lib().kvp_seq_append_token(self.handle, int(token)))
+
+    def reserve(self, num_tokens: int):
+        _check(lib().kvp_seq_reserve(self.handle, num_tokens))
+
+    def commit(self, new_tokens: int):
+        _check(lib().kvp_seq_commit(self.handle, new_tokens))
+
+    def free(self):
+        _check(lib().kvp_seq_free(self.handle))
+
+    def __len__(self) -> int:
+        return lib().kvp_seq_len(self.handle)
+
+    def num_blocks(self) -> int:
+        return lib().kvp_seq_num_blocks(self.handle)
+
+    def block_table(self, layer: int = 0, max_blocks: Optional[int] = None):
+        """(block ids, owned flags) of one layer; ids padded with -1 to max_blocks."""
+        n = self.num_blocks() if max_blocks is None else max_blocks
+        ids = (C.c_int32 * max(n, 1))()
+        owned = (C.c_uint8 * max(n, 1))()
+        rc = lib().kvp_seq_block_table(self.handle, layer, ids, n, owned)
+        if rc < 0:
+            _check(rc)
+        return list(ids)[:n], [bool(x) for x in list(owned)[:n]]
+
+    def close(self):
+        if self.handle:
+            lib().kvp_seq_destroy(self.handle)
+            self.handle = None
