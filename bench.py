@@ -163,14 +163,16 @@ def oracle_step(orc, wl, seqs, threads):
     tok = wl.cu_q[seqs]
     pk = wl.pool_k[sp.layer].copy()
     pv = wl.pool_v[sp.layer].copy()
-    rope = orc.rope_table(float(np.float32(sp.theta)), sp.D, wl.max_seq_len) if sp.theta else None
+    rope = orc.rope_table(float(np.float32(sp.theta)), sp.D, wl.max_seq_len, sp.rope_dim) if sp.theta else None
     st, q_out = orc.kv_append(Hq=sp.Hq, Hkv=sp.Hkv, D=sp.D, bs=sp.bs, kv_dtype=sp.kv_dtype, q=wl.q[tok], k=wl.k[tok],
                               v=wl.v[tok], tok_req=wl.tok_req[tok], positions=wl.positions[tok],
                               block_tables=wl.block_tables, pool_k=pk, pool_v=pv, max_seq_len=wl.max_seq_len,
-                              q_norm_w=wl.q_norm_w, k_norm_w=wl.k_norm_w, eps=sp.eps, rope=rope)
+                              q_norm_w=wl.q_norm_w, k_norm_w=wl.k_norm_w, eps=sp.eps, rope=rope,
+                              rope_dim=sp.rope_dim, rope_style=sp.rope_style, window=sp.window)
     st2, out, _ = orc.paged_attention(Hq=sp.Hq, Hkv=sp.Hkv, D=sp.D, bs=sp.bs, kv_dtype=sp.kv_dtype,
                                       q=q_out.reshape(-1, sp.Hq, sp.D), q_seq=seqs, q_pos=wl.ctx[seqs] - 1,
-                                      block_tables=wl.block_tables, pool_k=pk, pool_v=pv, threads=threads)
+                                      block_tables=wl.block_tables, pool_k=pk, pool_v=pv, threads=threads,
+                                      window=sp.window)
     return st | st2
 
 

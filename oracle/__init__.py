@@ -61,10 +61,11 @@ def lib():
                 "orc_rmsnorm_row": (None, [P, P, i32, f32, P]),
                 "orc_rope_table": (None, [f64, i32, i32, P]),
                 "orc_rope_row": (None, [P, i32, P, P]),
+                "orc_rope_row_ex": (None, [P, i32, i32, i32, P, P]),
                 "orc_kv_append": (i32, [i32, i32, i32, i32, i32, i32, i32, i32, i32,
-                                        P, P, P, P, P, f32, P, i32, P, P, P, i32, P, P, P]),
+                                        P, P, P, P, P, f32, P, i32, i32, i32, i32, P, P, P, i32, P, P, P]),
                 "orc_paged_attention": (i32, [i32, i32, i32, i32, i32, i32, i32, P, P, P, P, i32,
-                                              P, P, P, P, i32, i32]),
+                                              P, P, P, P, i32, i32, i32]),
                 "orc_gather_contiguous": (i32, [i32, i32, i32, i32, i32, P, i32, P, P]),
                 "orc_dense_attention": (i32, [i32, i32, i32, i32, P, i32, P, P, P]),
                 "orc_softmax_scale": (f64, [i32]),
@@ -123,18 +124,22 @@ def rmsnorm_row(x: np.ndarray, w: Optional[np.ndarray], eps: float) -> np.ndarra
     return y
 
 
-def rope_table(theta: float, D: int, max_pos: int) -> np.ndarray:
-    """[max_pos, D/2, 2] float32 (cos, sin)."""
-    t = np.empty((max_pos, D // 2, 2), dtype=np.float32)
-    lib().orc_rope_table(float(theta), D, max_pos, _p(t))
+def rope_table(theta: float, D: int, max_pos: int, rope_dim: int = 0) -> np.ndarray:
+    """[max_pos, R/2, 2] float32 (cos, sin) for the rotary width R = rope_dim
+    (0: D)."""
+    R = rope_dim or D
+    t = np.empty((max_pos, R // 2, 2), dtype=np.float32)
+    lib().orc_rope_table(float(theta), R, max_pos, _p(t))
     return t
 
 
-def rope_row(x: np.ndarray, cs: np.ndarray) -> np.ndarray:
+def rope_row(x: np.ndarray, cs: np.ndarray, rope_dim: int = 0, style: int = 0) -> np.ndarray:
+    """Rotates the first rope_dim dims (0: all) of one row; style 0 pairs
+    (i, i + rope_dim/2), style 1 pairs (2i, 2i + 1)."""
     x = _c(x, np.float32)
     cs = _c(cs, np.float32)
     y = np.empty_like(x)
-    lib().orc_rope_row(_p(x), x.size, _p(cs), _p(y))
+    lib().orc_rope_row_ex(_p(x), x.size, rope_dim or x.size, style, _p(cs), _p(y))
     return y
 
 
@@ -142,11 +147,14 @@ def rope_row(x: np.ndarray, cs: np.ndarray) -> np.ndarray:
 # kv_append / attention
 # --------------------------------------------------------------------------
 def kv_append(*, Hq, Hkv, D, bs, kv_dtype, q, k, v, tok_req, positions, block_tables, pool_k, pool_v,
-              max_seq_len, q_norm_w=None, k_norm_w=None, eps=1e-6, rope=None, S=None):
+              max_seq_len, q_norm_w=None, k_norm_w=None, eps=1e-6, rope=None, S=None, rope_dim=0,
+              rope_style=0, window=0):
     """Appends T tokens into ONE layer's pools (modified in place).
 
     pool_k / pool_v: uint16 [num_blocks, Hkv, bs, D], C-contiguous.
-    rope: [max_pos, D/2, 2] float32 table or None. Returns (status, q_out)."""
+    rope: [max_pos, R/2, 2] float32 table (R = rope_dim or D) or None.
+    window > 0: block-table rows are rings (entry (p / bs) mod row length).
+    Returns (status, q_out)."""
     q, k, v = _c(q, np.float32), _c(k, np.float32), _c(v, np.float32)
     T = len(tok_req)
     bt = _c(block_tables, np.int32)
@@ -159,16 +167,17 @@ def kv_append(*, Hq, Hkv, D, bs, kv_dtype, q, k, v, tok_req, positions, block_ta
     st = lib().orc_kv_append(
         T, S, Hq, Hkv, D, bs, nb, max_seq_len, DTYPES[kv_dtype], _p(q), _p(k), _p(v),
         _p(_c(q_norm_w, np.float32)), _p(_c(k_norm_w, np.float32)), eps,
-        _p(rope), 0 if rope is None else rope.shape[0],
+        _p(rope), 0 if rope is None else rope.shape[0], rope_dim, rope_style, window,
         _p(_c(tok_req, np.int32)), _p(_c(positions, np.int32)), _p(bt), bt.shape[1],
         _p(pool_k), _p(pool_v), _p(q_out))
     return st, q_out
 
 
 def paged_attention(*, Hq, Hkv, D, bs, kv_dtype, q, q_seq, q_pos, block_tables, pool_k, pool_v,
-                    want_weights=False, threads=0):
+                    want_weights=False, threads=0, window=0):
     """q: [NQ, Hq, D] float32; query i of sequence q_seq[i] at position q_pos[i]
-    sees keys 0..q_pos[i]. Returns (status, out [NQ,Hq,D] float32, weights)."""
+    sees keys 0..q_pos[i] (window > 0: the last `window` of them, through the
+    ring). Returns (status, out [NQ,Hq,D] float32, weights)."""
     q = _c(q, np.float32).reshape(-1, Hq, D)
     NQ = q.shape[0]
     q_seq, q_pos = _c(q_seq, np.int32), _c(q_pos, np.int32)
@@ -178,7 +187,7 @@ def paged_attention(*, Hq, Hkv, D, bs, kv_dtype, q, q_seq, q_pos, block_tables, 
     w = np.zeros((NQ, Hq, max(maxk, 1)), dtype=np.float64) if want_weights else None
     st = lib().orc_paged_attention(NQ, Hq, Hkv, D, bs, pool_k.shape[0], DTYPES[kv_dtype], _p(q), _p(q_seq),
                                    _p(q_pos), _p(bt), bt.shape[1], _p(pool_k), _p(pool_v), _p(out), _p(w),
-                                   max(maxk, 1), threads)
+                                   max(maxk, 1), window, threads)
     return st, out, w
 
 
@@ -211,11 +220,12 @@ def workload_append(wl, pool_k=None, pool_v=None):
     sp = wl.spec
     pk = wl.pool_k[sp.layer].copy() if pool_k is None else pool_k
     pv = wl.pool_v[sp.layer].copy() if pool_v is None else pool_v
-    rope = rope_table(sp.theta, sp.D, wl.max_seq_len) if sp.theta else None
+    rope = rope_table(sp.theta, sp.D, wl.max_seq_len, sp.rope_dim) if sp.theta else None
     st, q_out = kv_append(Hq=sp.Hq, Hkv=sp.Hkv, D=sp.D, bs=sp.bs, kv_dtype=sp.kv_dtype, q=wl.q, k=wl.k, v=wl.v,
                           tok_req=wl.tok_req, positions=wl.positions, block_tables=wl.block_tables,
                           pool_k=pk, pool_v=pv, max_seq_len=wl.max_seq_len, q_norm_w=wl.q_norm_w,
-                          k_norm_w=wl.k_norm_w, eps=sp.eps, rope=rope)
+                          k_norm_w=wl.k_norm_w, eps=sp.eps, rope=rope, rope_dim=sp.rope_dim,
+                          rope_style=sp.rope_style, window=sp.window)
     return st, q_out, pk, pv
 
 

@@ -31,10 +31,12 @@
  *
  * Readings where the pages are silent: NaN conversion keeps the payload's top bits and sets the quiet bit;
  * RMSNorm sums squares sequentially in fp32 and applies the weight after the
- * normalisation; RoPE is rotate-half (dims i and i+D/2) with angle
- * p * theta^(-2i/D), cos/sin evaluated in fp64 and rounded to fp32; a query at
- * position p sees keys 0..p; attention accumulates in fp64 from the exact
- * values of the stored 16-bit keys and values.
+ * normalisation; RoPE rotates the first rope_dim dims (all by default) as
+ * rotate-half pairs (i, i + rope_dim/2) or interleaved pairs (2i, 2i+1), with
+ * angle p * theta^(-2i/rope_dim), cos/sin evaluated in fp64 and rounded to
+ * fp32; a query at position p sees keys 0..p, or the last `window` of them
+ * read through a ring of block-table entries; attention accumulates in fp64
+ * from the exact values of the stored 16-bit keys and values.
  */
 #include <math.h>
 #include <stdint.h>
@@ -183,16 +185,19 @@ void orc_rmsnorm_row(const float *x, const float *w, int D, float eps, float *y)
 }
 
 /* ------------------------------------------------------------------------ */
-/* RoPE (reading: rotate-half pairs (i, i + D/2), angle p * theta^(-2i/D))   */
+/* RoPE (reading: pairs of the first rope_dim dims, angle p * theta^(-2i/rope_dim)) */
 /* ------------------------------------------------------------------------ */
 
-/* table[p][i] = (cos, sin) of p * theta^(-2i/D), fp64 rounded to fp32. */
-void orc_rope_table(double theta, int D, int max_pos, float *table)
+/* table[p][i] = (cos, sin) of p * theta^(-2i/R), i < R/2, fp64 rounded to fp32,
+ * for a rotary width R (R = head_dim for full rotary; the rope_dim of a
+ * partial-rotary layer, Op::Rope's rope_dim in the per-layer RoPE step of
+ * forward_layer in soft3/glia/run/arch/decoder/forward.rs). */
+void orc_rope_table(double theta, int R, int max_pos, float *table)
 {
-    int half = D / 2;
+    int half = R / 2;
     for (int p = 0; p < max_pos; ++p) {
         for (int i = 0; i < half; ++i) {
-            double inv_freq = pow(theta, -(2.0 * (double)i) / (double)D);
+            double inv_freq = pow(theta, -(2.0 * (double)i) / (double)R);
             double ang = (double)p * inv_freq;
             table[((int64_t)p * half + i) * 2 + 0] = (float)cos(ang);
             table[((int64_t)p * half + i) * 2 + 1] = (float)sin(ang);
@@ -200,18 +205,28 @@ void orc_rope_table(double theta, int D, int max_pos, float *table)
     }
 }
 
-/* Rotates one head row by the (cos, sin) pairs cs[i] of one position. */
-void orc_rope_row(const float *x, int D, const float *cs, float *y)
+/* Rotates one head row of D dims by the (cos, sin) pairs cs[i] of one
+ * position. Only the first R dims rotate (partial rotary); the rest are
+ * copied. Pair i is (i, i + R/2) for style 0 (rotate-half) and (2i, 2i + 1)
+ * for style 1 (interleaved); either way
+ *   y[a] = x[a]*c - x[b]*s,  y[b] = x[b]*c + x[a]*s,
+ * every product and sum rounded to fp32 separately. */
+void orc_rope_row_ex(const float *x, int D, int R, int style, const float *cs, float *y)
 {
-    int half = D / 2;
+    int half = R / 2;
+    for (int d = R; d < D; ++d) y[d] = x[d];
     for (int i = 0; i < half; ++i) {
+        int a = style ? 2 * i : i, b = style ? 2 * i + 1 : i + half;
         float c = cs[2 * i], s = cs[2 * i + 1];
-        float a = x[i], b = x[i + half];
-        float ac = a * c, bs = b * s, bc = b * c, as = a * s;
-        y[i] = ac - bs;
-        y[i + half] = bc + as;
+        float xa = x[a], xb = x[b];
+        float ac = xa * c, bs = xb * s, bc = xb * c, as = xa * s;
+        y[a] = ac - bs;
+        y[b] = bc + as;
     }
 }
+
+/* Full rotary, rotate-half. */
+void orc_rope_row(const float *x, int D, const float *cs, float *y) { orc_rope_row_ex(x, D, D, 0, cs, y); }
 
 /* ------------------------------------------------------------------------ */
 /* kv_append                                                                 */
@@ -224,24 +239,39 @@ static int64_t slot_index(int blk, int h, int slot, int d, int Hkv, int bs, int 
     return (((int64_t)blk * Hkv + h) * bs + slot) * D + d;
 }
 
+/* Block-table entry holding position p. With a sliding window (window > 0)
+ * a row is a ring of mbps blocks, the paged form of the window-sized ring
+ * cache of a sliding layer (kv_slot = past_seq_len % cache_seq in
+ * forward_layer, soft3/glia/run/arch/decoder/forward.rs): position p lives in
+ * entry (p / bs) mod mbps, slot p % bs. Without a window the entry is p / bs. */
+static int entry_of(int p, int bs, int mbps, int window)
+{
+    return window > 0 ? (p / bs) % mbps : p / bs;
+}
+
 /*
  * For each new token t of sequence r = tok_req[t] at position p = positions[t]:
- *   q' = rope(norm_q(q)), k' = rope(norm_k(k)), v' = v   (norm/rope optional)
- *   K/V slot = (block_tables[r][p / bs], p % bs); store convert(k'), convert(v')
+ *   q' = rope(norm_q(q)), k' = rope(norm_k(k)), v' = v   (norm/rope optional;
+ *        rope over the first rope_dim dims, pairing by rope_style)
+ *   K/V slot = (block_tables[r][entry_of(p)], p % bs); store convert(k'), convert(v')
  *   q_out[t] = q'
  * Rejected tokens (first error code returned):
+ *   window > 0 with mbps * bs < window -> ORC_EINVAL for the call, nothing done
  *   r outside [0, S)                   -> ORC_EINVAL, q_out row zeroed
  *   p outside [0, max_seq_len) or past the rope table
  *                                      -> ORC_EOVERFLOW, q_out row zeroed
- *   p / bs >= max_blocks_per_seq, or a block id outside [0, num_blocks)
+ *   entry >= max_blocks_per_seq, or a block id outside [0, num_blocks)
  *                                      -> ORC_ERANGE, q_out written, no store
  */
 int orc_kv_append(int T, int S, int Hq, int Hkv, int D, int bs, int num_blocks, int max_seq_len, int dtype,
                   const float *q, const float *k, const float *v, const float *q_norm_w, const float *k_norm_w,
-                  float eps, const float *rope, int rope_max_pos, const int32_t *tok_req, const int32_t *positions,
-                  const int32_t *block_tables, int mbps, uint16_t *pool_k, uint16_t *pool_v, float *q_out)
+                  float eps, const float *rope, int rope_max_pos, int rope_dim, int rope_style, int window,
+                  const int32_t *tok_req, const int32_t *positions, const int32_t *block_tables, int mbps,
+                  uint16_t *pool_k, uint16_t *pool_v, float *q_out)
 {
     int status = ORC_OK;
+    if (rope_dim == 0) rope_dim = D;
+    if (window > 0 && (int64_t)mbps * bs < window) return ORC_EINVAL;
     float *t0 = malloc(sizeof(float) * D), *t1 = malloc(sizeof(float) * D);
 #define ORC_FAIL(code) do { if (status == ORC_OK) status = (code); } while (0)
     for (int t = 0; t < T; ++t) {
@@ -257,15 +287,15 @@ int orc_kv_append(int T, int S, int Hq, int Hkv, int D, int bs, int num_blocks, 
             memset(qo, 0, sizeof(float) * Hq * D);
             continue;
         }
-        const float *cs = rope ? rope + (int64_t)p * D : NULL; /* D/2 pairs */
+        const float *cs = rope ? rope + (int64_t)p * rope_dim : NULL; /* rope_dim/2 pairs */
         for (int g = 0; g < Hq; ++g) {
             const float *x = q + ((int64_t)t * Hq + g) * D;
             memcpy(t0, x, sizeof(float) * D);
             if (q_norm_w) { orc_rmsnorm_row(t0, q_norm_w, D, eps, t1); memcpy(t0, t1, sizeof(float) * D); }
-            if (cs) { orc_rope_row(t0, D, cs, t1); memcpy(t0, t1, sizeof(float) * D); }
+            if (cs) { orc_rope_row_ex(t0, D, rope_dim, rope_style, cs, t1); memcpy(t0, t1, sizeof(float) * D); }
             memcpy(qo + (int64_t)g * D, t0, sizeof(float) * D);
         }
-        int j = p / bs, slot = p % bs;
+        int j = entry_of(p, bs, mbps, window), slot = p % bs;
         if (j >= mbps) { ORC_FAIL(ORC_ERANGE); continue; }
         int blk = block_tables[(int64_t)r * mbps + j];
         if (blk < 0 || blk >= num_blocks) { ORC_FAIL(ORC_ERANGE); continue; }
@@ -273,7 +303,7 @@ int orc_kv_append(int T, int S, int Hq, int Hkv, int D, int bs, int num_blocks, 
             const float *x = k + ((int64_t)t * Hkv + h) * D;
             memcpy(t0, x, sizeof(float) * D);
             if (k_norm_w) { orc_rmsnorm_row(t0, k_norm_w, D, eps, t1); memcpy(t0, t1, sizeof(float) * D); }
-            if (cs) { orc_rope_row(t0, D, cs, t1); memcpy(t0, t1, sizeof(float) * D); }
+            if (cs) { orc_rope_row_ex(t0, D, rope_dim, rope_style, cs, t1); memcpy(t0, t1, sizeof(float) * D); }
             const float *vx = v + ((int64_t)t * Hkv + h) * D;
             for (int d = 0; d < D; ++d) {
                 uint32_t kb, vb;
@@ -301,25 +331,30 @@ typedef struct {
     const uint16_t *k, *v;
     const int32_t *bt; /* paged: this sequence's block table row */
     int paged, Hkv, bs, D, h, dtype;
+    int mbps, window;  /* paged: entry_of's ring when window > 0 */
 } kv_src;
 
 static const uint16_t *key_row(const kv_src *s, int j, const uint16_t *base)
 {
     if (s->paged)
-        return base + slot_index(s->bt[j / s->bs], s->h, j % s->bs, 0, s->Hkv, s->bs, s->D);
+        return base + slot_index(s->bt[entry_of(j, s->bs, s->mbps, s->window)], s->h, j % s->bs, 0, s->Hkv, s->bs,
+                                 s->D);
     return base + ((int64_t)j * s->Hkv + s->h) * s->D; /* contiguous [nk][Hkv][D] */
 }
 
-static void attend_one(const float *qrow, int nk, const kv_src *src, double scale, double *sbuf, float *out,
+/* One query head over keys j0 .. nk-1 (sbuf holds nk doubles; w_out, if
+ * given, receives weight j at index j and 0 below j0). */
+static void attend_one(const float *qrow, int j0, int nk, const kv_src *src, double scale, double *sbuf, float *out,
                        double *w_out)
 {
     int D = src->D;
-    if (nk <= 0) {
+    if (nk <= j0) {
         for (int d = 0; d < D; ++d) out[d] = 0.0f;
         return;
     }
+    for (int j = 0; j < j0; ++j) sbuf[j] = 0.0;
     double m = -INFINITY;
-    for (int j = 0; j < nk; ++j) {
+    for (int j = j0; j < nk; ++j) {
         const uint16_t *kr = key_row(src, j, src->k);
         double acc = 0.0;
         for (int d = 0; d < D; ++d)
@@ -328,14 +363,14 @@ static void attend_one(const float *qrow, int nk, const kv_src *src, double scal
         if (sbuf[j] > m) m = sbuf[j];
     }
     double l = 0.0;
-    for (int j = 0; j < nk; ++j) {
+    for (int j = j0; j < nk; ++j) {
         sbuf[j] = exp(sbuf[j] - m);
         l += sbuf[j];
     }
-    for (int j = 0; j < nk; ++j) sbuf[j] /= l;
+    for (int j = j0; j < nk; ++j) sbuf[j] /= l;
     if (w_out) memcpy(w_out, sbuf, sizeof(double) * nk);
     double *acc = calloc(D, sizeof(double));
-    for (int j = 0; j < nk; ++j) {
+    for (int j = j0; j < nk; ++j) {
         const uint16_t *vr = key_row(src, j, src->v);
         for (int d = 0; d < D; ++d) acc[d] += sbuf[j] * orc_value16(vr[d], src->dtype);
     }
@@ -348,18 +383,24 @@ double orc_softmax_scale(int D) { return (double)(float)(1.0 / sqrt((double)D));
 
 /*
  * Paged attention for NQ queries. Query i belongs to sequence q_seq[i], sits at
- * position q_pos[i] and sees keys 0..q_pos[i] of that sequence (q_pos = -1:
- * no keys, output zeros). q and out are [NQ][Hq][D] float32. Query head g
- * reads kv head g / (Hq / Hkv). weights (optional) receives the softmax
- * weights, [NQ][Hq][max_keys]. A block id outside [0, num_blocks) or a block
- * index past mbps zeroes that query's output and returns ORC_ERANGE.
+ * position p = q_pos[i] and sees keys 0..p of that sequence (q_pos = -1: no
+ * keys, output zeros); with a sliding window (window > 0) only keys
+ * max(0, p - window + 1)..p, read through entry_of's ring (the window of
+ * forward_layer in soft3/glia/run/arch/decoder/forward.rs: the last cache_seq
+ * positions, read_start = total_seq - cache_seq). q and out are [NQ][Hq][D]
+ * float32. Query head g reads kv head g / (Hq / Hkv). weights (optional)
+ * receives the softmax weights, [NQ][Hq][max_keys], indexed by key position.
+ * A block id outside [0, num_blocks) or a block index past mbps zeroes that
+ * query's output and returns ORC_ERANGE; window > 0 with mbps * bs < window
+ * returns ORC_EINVAL before any work.
  */
 int orc_paged_attention(int NQ, int Hq, int Hkv, int D, int bs, int num_blocks, int dtype, const float *q,
                         const int32_t *q_seq, const int32_t *q_pos, const int32_t *block_tables, int mbps,
                         const uint16_t *pool_k, const uint16_t *pool_v, float *out, double *weights, int max_keys,
-                        int threads)
+                        int window, int threads)
 {
     if (Hkv <= 0 || Hq % Hkv) return ORC_EUNSUPPORTED;
+    if (window > 0 && (int64_t)mbps * bs < window) return ORC_EINVAL;
     int group = Hq / Hkv, status = ORC_OK;
     double scale = orc_softmax_scale(D);
 #ifdef _OPENMP
@@ -368,10 +409,13 @@ int orc_paged_attention(int NQ, int Hq, int Hkv, int D, int bs, int num_blocks, 
 #pragma omp parallel for schedule(dynamic, 1)
     for (int i = 0; i < NQ; ++i) {
         int r = q_seq[i], nk = q_pos[i] + 1;
+        int j0 = window > 0 && nk > window ? nk - window : 0;
         const int32_t *bt = block_tables + (int64_t)r * mbps;
-        int bad = nk > mbps * bs;
-        for (int j = 0; !bad && j < nk; j += bs)
-            bad = bt[j / bs] < 0 || bt[j / bs] >= num_blocks;
+        int bad = window == 0 && nk > mbps * bs;
+        for (int j = j0; !bad && j < nk; ++j) {
+            int e = entry_of(j, bs, mbps, window);
+            bad = bt[e] < 0 || bt[e] >= num_blocks;
+        }
         if (bad) {
             memset(out + (int64_t)i * Hq * D, 0, sizeof(float) * Hq * D);
 #pragma omp critical
@@ -380,9 +424,10 @@ int orc_paged_attention(int NQ, int Hq, int Hkv, int D, int bs, int num_blocks, 
         }
         double *sbuf = malloc(sizeof(double) * (nk > 0 ? nk : 1));
         for (int g = 0; g < Hq; ++g) {
-            kv_src src = {pool_k, pool_v, bt, 1, Hkv, bs, D, g / group, dtype};
+            kv_src src = {pool_k, pool_v, bt, 1, Hkv, bs, D, g / group, dtype, mbps, window};
             double *w = weights ? weights + ((int64_t)i * Hq + g) * max_keys : NULL;
-            attend_one(q + ((int64_t)i * Hq + g) * D, nk, &src, scale, sbuf, out + ((int64_t)i * Hq + g) * D, w);
+            attend_one(q + ((int64_t)i * Hq + g) * D, j0, nk, &src, scale, sbuf, out + ((int64_t)i * Hq + g) * D,
+                       w);
         }
         free(sbuf);
     }
@@ -413,8 +458,8 @@ int orc_dense_attention(int Hq, int Hkv, int D, int dtype, const float *q, int n
     double *sbuf = malloc(sizeof(double) * (nk > 0 ? nk : 1));
     double scale = orc_softmax_scale(D);
     for (int g = 0; g < Hq; ++g) {
-        kv_src src = {ck, cv, NULL, 0, Hkv, 0, D, g / (Hq / Hkv), dtype};
-        attend_one(q + (int64_t)g * D, nk, &src, scale, sbuf, out + (int64_t)g * D, NULL);
+        kv_src src = {ck, cv, NULL, 0, Hkv, 0, D, g / (Hq / Hkv), dtype, 0, 0};
+        attend_one(q + (int64_t)g * D, 0, nk, &src, scale, sbuf, out + (int64_t)g * D, NULL);
     }
     free(sbuf);
     return ORC_OK;

@@ -100,7 +100,7 @@ def oracle_decode(orc, wl, q_out, pk, pv, seqs=None, threads=0):
     q = q_out[tok].reshape(-1, sp.Hq, sp.D)
     st, out, _ = orc.paged_attention(Hq=sp.Hq, Hkv=sp.Hkv, D=sp.D, bs=sp.bs, kv_dtype=sp.kv_dtype, q=q,
                                      q_seq=seqs, q_pos=wl.ctx[seqs] - 1, block_tables=wl.block_tables,
-                                     pool_k=pk, pool_v=pv, threads=threads)
+                                     pool_k=pk, pool_v=pv, threads=threads, window=sp.window)
     return st, out
 
 
@@ -111,7 +111,7 @@ def oracle_rows(orc, wl, q_out, pk, pv, rows, threads=0):
     st, out, _ = orc.paged_attention(Hq=sp.Hq, Hkv=sp.Hkv, D=sp.D, bs=sp.bs, kv_dtype=sp.kv_dtype,
                                      q=q_out[rows].reshape(-1, sp.Hq, sp.D), q_seq=wl.tok_req[rows],
                                      q_pos=wl.positions[rows], block_tables=wl.block_tables, pool_k=pk, pool_v=pv,
-                                     threads=threads)
+                                     threads=threads, window=sp.window)
     return st, out
 
 

@@ -136,7 +136,7 @@ def _decode(orc, wl, pk, pv, q=None):
     q = wl.q.reshape(-1, sp.Hq, sp.D) if q is None else q
     return orc.paged_attention(Hq=sp.Hq, Hkv=sp.Hkv, D=sp.D, bs=sp.bs, kv_dtype=sp.kv_dtype, q=q,
                                q_seq=wl.tok_req, q_pos=wl.positions, block_tables=wl.block_tables,
-                               pool_k=pk, pool_v=pv, want_weights=True)
+                               pool_k=pk, pool_v=pv, want_weights=True, window=sp.window)
 
 
 def test_attention_weights_sum_to_one_and_match_dense_twin(orc, wl_small):

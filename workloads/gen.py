@@ -31,6 +31,12 @@ write shows up as a changed sentinel.
 
 Pool layout (per layer): ``[num_blocks][Hkv][block_size][D]`` 16-bit words,
 head-major inside a block, so one (block, head) tile is contiguous.
+
+Sliding-window specs (``window > 0``) give every sequence a ring of
+``ring_blocks`` block-table entries (default ``ceil(window / block_size)``):
+position p lives in entry ``(p // block_size) % ring_blocks``, so only the
+last ``ring_blocks * block_size`` prior tokens are resident and drawn (in
+position order), each at its ring slot.
 """
 
 from __future__ import annotations
@@ -80,6 +86,10 @@ class Spec:
     num_layers: int = 1
     layer: int = 0
     seed_offset: int = 0
+    rope_dim: int = 0  # rotated leading dims (0: all D)
+    rope_style: int = 0  # 0: pairs (i, i + rope_dim/2); 1: pairs (2i, 2i + 1)
+    window: int = 0  # sliding window in keys (0: none); block-table rows become rings
+    ring_blocks: int = 0  # ring length in blocks (0: ceil(window / bs))
     description: str = ""
 
 
@@ -117,18 +127,26 @@ class Workload:
     def prefill_seqs(self) -> np.ndarray:
         return np.nonzero(self.q_lens > 1)[0].astype(np.int32)
 
+    def visible_keys(self, seqs: Optional[Sequence[int]] = None) -> np.ndarray:
+        """Keys the decode query of each sequence sees: its context, or the
+        last `window` of it."""
+        s = self.decode_seqs if seqs is None else np.asarray(seqs)
+        n = self.ctx[s].astype(np.int64)
+        return np.minimum(n, self.spec.window) if self.spec.window > 0 else n
+
     def kv_read_bytes(self, seqs: Optional[Sequence[int]] = None) -> int:
         """Algorithmic K+V bytes one decode pass reads: every visible key and
         value element once, for every KV head."""
-        s = self.decode_seqs if seqs is None else np.asarray(seqs)
         sp = self.spec
-        return int(self.ctx[s].astype(np.int64).sum()) * sp.Hkv * sp.D * 2 * 2
+        return int(self.visible_keys(seqs).sum()) * sp.Hkv * sp.D * 2 * 2
 
     def unique_kv_read_bytes(self, seqs: Optional[Sequence[int]] = None) -> int:
         """Like kv_read_bytes but counting each physical block slot once
         (shared prefix blocks are read by several sequences)."""
         s = self.decode_seqs if seqs is None else np.asarray(seqs)
         sp = self.spec
+        if sp.window > 0:  # rings are private
+            return self.kv_read_bytes(s)
         seen = {}
         for r in s:
             n = int(self.ctx[r])
@@ -185,6 +203,15 @@ def make_workload(spec: Spec, seed_offset: Optional[int] = None) -> Workload:
     ctx = prior + q_lens
     nblk = (ctx.astype(np.int64) + bs - 1) // bs
     mbps = int(max(1, nblk.max(initial=1)))
+    ring = 0
+    if spec.window > 0:
+        if spec.share_group:
+            raise ValueError("sliding-window rings are private: no prefix sharing")
+        ring = spec.ring_blocks or -(-spec.window // bs)
+        if ring * bs < spec.window:
+            raise ValueError("the ring must hold the window")
+        nblk = np.minimum(nblk, ring)
+        mbps = ring
 
     # sharing groups: sequence r shares its first n_shared[r] blocks
     share_blocks = spec.share_tokens // bs if spec.share_group else 0
@@ -242,6 +269,19 @@ def make_workload(spec: Spec, seed_offset: Optional[int] = None) -> Workload:
         # members with shorter priors use a prefix of the group's blocks
         _place(group_blocks[g], 0, kx, vx)
     for r in range(S):
+        if ring:
+            # the resident positions [max(0, prior - ring*bs), prior) at their ring slots
+            first = max(0, int(prior[r]) - ring * bs)
+            n = int(prior[r]) - first
+            if n <= 0:
+                continue
+            kx = _truncate_to_16(_normal(rng, (n, Hkv, D), spec.value_scale), spec.kv_dtype)
+            vx = _truncate_to_16(_normal(rng, (n, Hkv, D), spec.value_scale), spec.kv_dtype)
+            pos = np.arange(first, first + n)
+            ids = bt[r, (pos // bs) % ring]
+            pk[ids, :, pos % bs, :] = kx
+            pv[ids, :, pos % bs, :] = vx
+            continue
         start = int(n_shared[r]) * bs
         n = int(prior[r]) - start
         if n <= 0:
@@ -272,7 +312,7 @@ def make_workload(spec: Spec, seed_offset: Optional[int] = None) -> Workload:
     return Workload(
         spec=spec, S=S, prior=prior, q_lens=q_lens, ctx=ctx.astype(np.int32), cu_q=cu_q,
         max_blocks_per_seq=mbps, block_tables=bt, num_blocks=num_blocks,
-        max_seq_len=mbps * bs, T=T, tok_req=tok_req, positions=positions.astype(np.int32),
+        max_seq_len=max(mbps * bs, int(ctx.max(initial=0))), T=T, tok_req=tok_req, positions=positions.astype(np.int32),
         q=q, k=k, v=v, q_norm_w=qn, k_norm_w=kn, pool_k=pool_k, pool_v=pool_v,
         shared_blocks=share_blocks,
     )
@@ -307,6 +347,13 @@ SPECS = {
         segments=(Segment(q_len=1, fixed=(32768,) * 8),), value_scale=0.5, seed_offset=4,
         description="long-context decode, batch 8, GQA 8:1, D=128, bs=16, bf16, 32768 cached "
                     "tokens each, values x0.5",
+    ),
+    "mistral-swa-b32": Spec(
+        name="mistral-swa-b32", Hq=32, Hkv=8, D=128, bs=16, kv_dtype="bf16", theta=1e4,
+        segments=(Segment(q_len=1, count=32, prior_lo=2048, prior_hi=32768),), window=4096,
+        seed_offset=6,
+        description="Mistral-7B-shaped sliding-window decode, batch 32, Hq=32, Hkv=8, D=128, "
+                    "bs=16, bf16, context U[2048,32768], window 4096 over a ring of 256 blocks",
     ),
     "mixed-prefill": Spec(
         name="mixed-prefill", Hq=32, Hkv=8, D=128, bs=16, kv_dtype="f16", theta=5e5,
