@@ -253,8 +253,9 @@ def run_ours(args):
     pool = K.Pool(sp.num_layers, sp.Hkv, sp.D, sp.bs, wl.max_seq_len, wl.num_blocks, sp.kv_dtype, device=dev)
     pool.k.copy_(torch.from_numpy(wl.pool_k.view(np.int16)))
     pool.v.copy_(torch.from_numpy(wl.pool_v.view(np.int16)))
-    attn = K.attn_config(sp.Hq, sp.Hkv, sp.D, float(np.float32(sp.theta)), sp.eps)
-    rope = torch.empty(wl.max_seq_len * sp.D, dtype=torch.float32, device=dev)
+    attn = K.attn_config(sp.Hq, sp.Hkv, sp.D, float(np.float32(sp.theta)), sp.eps, sp.rope_dim, sp.rope_style,
+                         sp.window)
+    rope = torch.empty(wl.max_seq_len * (sp.rope_dim or sp.D), dtype=torch.float32, device=dev)
     K.rope_table_fill(attn, wl.max_seq_len, rope)
     g = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(dev)
     # the step's per-step inputs live in one device buffer (256-byte aligned
@@ -317,7 +318,10 @@ def run_ours(args):
                                                                device=dev)
         p_out = torch.empty_like(p_q)
         p_maxq = int(wl.q_lens[pseq].max())
-        pairs = int((wl.positions[p_rows].astype(np.int64) + 1).sum())  # causal (query, key) pairs
+        seen = wl.positions[p_rows].astype(np.int64) + 1  # causal (query, key) pairs
+        if sp.window > 0:
+            seen = np.minimum(seen, sp.window)
+        pairs = int(seen.sum())
         prefill_flops = pairs * sp.Hq * sp.D * 4  # QK^T and PV, 2 flops per multiply-add
 
     def append():

@@ -89,13 +89,37 @@ typedef struct {
  * HeadDim, RopeTheta) of makarna/pkg/model/arch/hybrid_decoder.go plus the
  * q/k RMSNorm epsilon. num_kv_heads == 0 means num_heads
  * (normalizeHybridDecoderConfig). num_heads / num_kv_heads (the GQA group)
- * must be 1, 2, 4 or 8 for the decode path. */
+ * must be 1, 2, 4 or 8 for the decode path.
+ *
+ * The last three fields are those of a per-layer RoPE and cache (the
+ * layer_rope_dim / layer_kv_cache_seq of forward_layer in
+ * soft3/glia/run/arch/decoder/forward.rs); zero-filled they give full
+ * rotate-half RoPE and unlimited attention:
+ *   rope_dim   rotated leading dims: 0 = head_dim, else even and <= head_dim;
+ *              the rest of the row passes through unrotated
+ *   rope_style KVP_ROPE_HALF: pairs (i, i + rope_dim/2);
+ *              KVP_ROPE_INTERLEAVED: pairs (2i, 2i + 1)
+ *   window     0, or a sliding window: the query at position p sees keys
+ *              max(0, p - window + 1) .. p only, and every block-table row is
+ *              a RING of max_blocks_per_seq entries -- position p lives in
+ *              entry (p / block_size) mod max_blocks_per_seq, slot
+ *              p % block_size (the paged form of a sliding layer's
+ *              window-sized ring cache, kv_slot = past_seq_len % cache_seq).
+ *              Calls refuse max_blocks_per_seq * block_size < window with
+ *              KVP_EINVAL. A position's slot is reused once the position has
+ *              left every window, so positions past
+ *              max_blocks_per_seq * block_size are accepted (up to
+ *              max_seq_len). */
+enum { KVP_ROPE_HALF = 0, KVP_ROPE_INTERLEAVED = 1 };
 typedef struct {
     int32_t num_heads;
     int32_t num_kv_heads;
     int32_t head_dim;
     float rope_theta;
     float rms_eps;
+    int32_t rope_dim;
+    int32_t rope_style;
+    int32_t window;
 } kvp_attn_config;
 
 typedef struct kvp_pool kvp_pool; /* opaque host handle */
@@ -129,14 +153,15 @@ const char *kvp_last_error(void);
 /* Size in bytes of a RoPE table covering positions [0, max_pos). */
 size_t kvp_rope_table_bytes(const kvp_attn_config *attn, int max_pos);
 
-/* Fills a caller-owned DEVICE table [max_pos][head_dim/2] of (cos, sin)
- * float pairs for rotate-half RoPE: pair i at position p rotates dims
- * (i, i + D/2) by the angle p * theta^(-2i/D), evaluated in fp64 and rounded
- * to fp32. The pages leave HybridRoPE's formula unstated; this is the
- * rotate-half convention of the Llama-3 / Qwen3 shapes they serve. Computed
- * once at set-up time on the host and copied with a blocking cudaMemcpy:
- * call it outside any stream capture. theta must be > 0, head_dim even and
- * <= 256 (the fused-RoPE limits of runHybridAttentionBlock). */
+/* Fills a caller-owned DEVICE table [max_pos][R/2] of (cos, sin) float
+ * pairs, R = the config's rotary width (rope_dim, or head_dim when 0): pair i
+ * at position p rotates by the angle p * theta^(-2i/R), evaluated in fp64 and
+ * rounded to fp32. The pages leave HybridRoPE's formula unstated; by default
+ * this is the rotate-half convention of the Llama-3 / Qwen3 shapes they
+ * serve (rope_style picks the dims a pair turns). Computed once at set-up
+ * time on the host and copied with a blocking cudaMemcpy: call it outside
+ * any stream capture. theta must be > 0, head_dim even and <= 256 (the
+ * fused-RoPE limits of runHybridAttentionBlock). */
 int kvp_rope_table_fill(const kvp_attn_config *attn, int max_pos, float *table);
 
 /* ------------------------------------------------------------ kv_append */
@@ -147,14 +172,17 @@ int kvp_rope_table_fill(const kvp_attn_config *attn, int max_pos, float *table);
  *
  * For token t of sequence r = tok_req[t] at position p = positions[t]:
  *   q' = rope(norm(q[t], q_norm_w)),  k' = rope(norm(k[t], k_norm_w)),  v' = v[t]
- *   the K/V slot is (block_tables[r][p / block_size], p % block_size);
+ *   the K/V slot is (block_tables[r][p / block_size], p % block_size), or
+ *   with a window entry (p / block_size) mod max_blocks_per_seq (the ring);
  *   K and V receive cvt(k'), cvt(v') with cvt = nearest 16-bit value, ties to
  *   even (float32ToFloat16Bits / float32ToBFloat16Bits; a NaN becomes a quiet
  *   NaN keeping its top payload bits); q_out[t] = q'.
  * norm(x, w) = (x * (1 / sqrt(sum_d x_d^2 * (1/D) + eps))) * w with the sum
  * taken in order d = 0..D-1 in fp32 (the per-head RMS form of forward_layer in
  * soft3/glia/run/arch/decoder/forward.rs); skipped when the weight is NULL.
- * rope uses the table of kvp_rope_table_fill; skipped when rope_table is NULL.
+ * rope uses the table of kvp_rope_table_fill (built for the same rope_dim)
+ * on the first rope_dim dims, paired as rope_style says; skipped when
+ * rope_table is NULL.
  * Every float step is one IEEE operation, so results are reproducible bit for
  * bit.
  *
@@ -165,9 +193,10 @@ int kvp_rope_table_fill(const kvp_attn_config *attn, int max_pos, float *table);
  *   q_out      [T][Hq][D] float32 (written for every accepted token)
  * Device errors: tok_req outside [0, num_seqs) -> KVP_EINVAL; position outside
  * [0, max_seq_len) or past the rope table -> KVP_EOVERFLOW (q_out row zeroed);
- * p / block_size >= max_blocks_per_seq or a block id outside [0, num_blocks)
- * -> KVP_ERANGE (q_out still written, no store). Two tokens aimed at the same
- * slot in one call race. T == 0 is a no-op. */
+ * p / block_size >= max_blocks_per_seq (without a window) or a block id
+ * outside [0, num_blocks) -> KVP_ERANGE (q_out still written, no store). Two
+ * tokens aimed at the same slot in one call race (with a ring: two positions
+ * of one sequence max_blocks_per_seq * block_size apart). T == 0 is a no-op. */
 int kv_append(kvp_pool *pool, int layer, const kvp_attn_config *attn, int T, const float *q, const float *k,
               const float *v, const float *q_norm_w, const float *k_norm_w, const float *rope_table,
               int rope_max_pos, const int32_t *tok_req, const int32_t *positions, int num_seqs,
@@ -185,8 +214,9 @@ size_t paged_decode_workspace_size(const kvp_pool *pool, const kvp_attn_config *
  * runHybridAttentionBlockBatch in makarna/pkg/model/arch/hybrid_decoder.go;
  * the attention of forward_layer in soft3/glia/run/arch/decoder/forward.rs).
  * Query head g of sequence r reads KV head g / (Hq/Hkv) and the keys
- * 0 .. ctx_lens[r]-1, i.e. ctx_lens[r] counts the cached keys INCLUDING the
- * token kv_append just wrote:
+ * 0 .. ctx_lens[r]-1 (with a window, the last `window` of them, through the
+ * ring), i.e. ctx_lens[r] counts the keys INCLUDING the token kv_append just
+ * wrote:
  *   out[r][g] = sum_j softmax_j(q[r][g] . K_j * scale) V_j,
  *   scale = float32(1/sqrt(float64(D))),
  * accumulated in fp32 with an online softmax over 16-key tiles. The tiles of
@@ -208,9 +238,9 @@ size_t paged_decode_workspace_size(const kvp_pool *pool, const kvp_attn_config *
  *                 aligned, ZERO-FILLED before its first use; every call leaves
  *                 its counters at zero again. Calls sharing a workspace must
  *                 not overlap on the device.
- * Device errors: ctx_lens[r] above max_ctx_len, max_blocks_per_seq*block_size
- * or max_seq_len -> KVP_ERANGE and a zero row; a block id outside the pool ->
- * KVP_ERANGE and that block is left out. */
+ * Device errors: ctx_lens[r] above max_ctx_len, max_seq_len or (without a
+ * window) max_blocks_per_seq*block_size -> KVP_ERANGE and a zero row; a block
+ * id outside the pool -> KVP_ERANGE and that block is left out. */
 int paged_decode_attention(kvp_pool *pool, int layer, const kvp_attn_config *attn, int B, const float *q,
                            const int32_t *block_tables, int max_blocks_per_seq, const int32_t *ctx_lens,
                            int max_ctx_len, int split_tokens, float *out, void *workspace, size_t ws_bytes,
@@ -254,13 +284,23 @@ size_t paged_prefill_workspace_size(const kvp_pool *pool, const kvp_attn_config 
  * runHybridAttentionBlock for seqLen > 1, with kvLen = startPos + seqLen).
  * Sequence s has q_len_s = cu_q[s+1] - cu_q[s] >= 1 new queries whose K/V
  * kv_append already wrote; its query i sits at position
- * ctx_lens[s] - q_len_s + i and sees keys 0 .. that position (causal).
+ * ctx_lens[s] - q_len_s + i and sees keys 0 .. that position (causal), or
+ * with a window the last `window` of them. With a window the chunk must not
+ * have overwritten, in its ring, a key one of its own queries needs: a
+ * sequence whose smallest needed key max(0, ctx - q_len - window + 1) is at
+ * or below ctx - 1 - max_blocks_per_seq * block_size is refused (append such a
+ * chunk in pieces of at most max_blocks_per_seq * block_size - window + 1
+ * tokens, attending after each).
  *   q, out   [total_q][Hq][D] float32 (rows cu_q[s] .. cu_q[s+1]-1 belong to s)
  *   cu_q     [S+1] int32, cu_q[0] = 0, cu_q[S] = total_q; max_q_len bounds q_len_s
  *   ctx_lens [S] int32; block_tables [S][max_blocks_per_seq]
- * QK^T and PV run on the tensor cores with fp16 operands (q and the softmax
- * weights rounded to fp16) and fp32 accumulation; the softmax is fp32.
- * Device errors as paged_decode_attention. */
+ * QK^T and PV run on the tensor cores with 16-bit operands of the pool's type
+ * (q and the softmax weights rounded to it; K and V exact) and fp32
+ * accumulation; the softmax is fp32. With an fp16 pool the outputs agree with
+ * exact attention within 1e-3 + 1e-3*|x|; with a bf16 pool (8 significant
+ * bits) within about 1e-2 + 1e-2*|x|.
+ * Device errors as paged_decode_attention, plus KVP_ERANGE for a refused
+ * sequence (its rows are left unwritten). */
 int paged_prefill_attention(kvp_pool *pool, int layer, const kvp_attn_config *attn, int S, const float *q,
                             const int32_t *cu_q, const int32_t *ctx_lens, const int32_t *block_tables,
                             int max_blocks_per_seq, int total_q, int max_q_len, float *out, void *workspace,

@@ -14,6 +14,8 @@ from ._native import (  # noqa: F401
     KVP_EUNSUPPORTED,
     KVP_F16,
     KVP_OK,
+    KVP_ROPE_HALF,
+    KVP_ROPE_INTERLEAVED,
     AttnConfig,
     Blocks,
     CacheConfig,

@@ -51,7 +51,11 @@ class CacheConfig(C.Structure):
 
 class AttnConfig(C.Structure):
     _fields_ = [("num_heads", C.c_int32), ("num_kv_heads", C.c_int32), ("head_dim", C.c_int32),
-                ("rope_theta", C.c_float), ("rms_eps", C.c_float)]
+                ("rope_theta", C.c_float), ("rms_eps", C.c_float), ("rope_dim", C.c_int32),
+                ("rope_style", C.c_int32), ("window", C.c_int32)]
+
+
+KVP_ROPE_HALF, KVP_ROPE_INTERLEAVED = 0, 1
 
 
 _lib = None
@@ -127,8 +131,12 @@ def _stream(stream) -> C.c_void_p:
 
 
 def attn_config(num_heads: int, num_kv_heads: int, head_dim: int, rope_theta: float = 0.0,
-                rms_eps: float = 1e-6) -> AttnConfig:
-    return AttnConfig(num_heads, num_kv_heads, head_dim, rope_theta, rms_eps)
+                rms_eps: float = 1e-6, rope_dim: int = 0, rope_style: int = KVP_ROPE_HALF,
+                window: int = 0) -> AttnConfig:
+    """rope_dim: rotated leading dims (0: all); rope_style: KVP_ROPE_HALF or
+    KVP_ROPE_INTERLEAVED; window > 0: sliding window, block-table rows are
+    rings of their length."""
+    return AttnConfig(num_heads, num_kv_heads, head_dim, rope_theta, rms_eps, rope_dim, rope_style, window)
 
 
 class Pool:

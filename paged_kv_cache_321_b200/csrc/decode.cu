@@ -100,6 +100,7 @@ struct Params {
     int *counters;            // [B*Hkv] segments finished per split context
     int *status;
     int B, Hq, Hkv, mbps, bs, num_blocks, max_ctx, max_seq_len, warps_total, min_tiles;
+    int window;    // sliding window in keys (0: none); > 0 makes block-table rows rings
     float qscale;  // softmax scale * log2(e)
 };
 
@@ -201,7 +202,7 @@ struct Cursor {
 // reported by the decode kernel).
 __device__ __forceinline__ bool ctx_ok(const Params &p, int c)
 {
-    return c >= 0 && c <= p.max_ctx && c <= p.mbps * p.bs && c <= p.max_seq_len;
+    return c >= 0 && c <= p.max_ctx && c <= p.max_seq_len && (p.window > 0 || c <= p.mbps * p.bs);
 }
 
 // Cost of starting a context on a warp, in tiles: a warp whose range crosses
@@ -212,19 +213,42 @@ __device__ __forceinline__ bool ctx_ok(const Params &p, int c)
 constexpr int kCtxCost = 1;
 
 // The kernels keep each sequence's context length in shared memory (-1 for
-// one the kernel refuses), and derive its number of tiles from it.
-__device__ __forceinline__ int tiles_of(int ctx) { return ctx > 0 ? (ctx + TT - 1) / TT : 0; }
+// one the kernel refuses), and derive its tiles from it: the keys of a
+// context are 0 .. ctx-1, or with a sliding window ctx-window .. ctx-1,
+// covered by the 16-key tiles first_tile .. (ctx-1)/16 of the position axis.
+__device__ __forceinline__ int first_tile(int ctx, int window)
+{
+    return window > 0 && ctx > window ? (ctx - window) / TT : 0;
+}
+__device__ __forceinline__ int tiles_of(int ctx, int window)
+{
+    return ctx > 0 ? (ctx + TT - 1) / TT - first_tile(ctx, window) : 0;
+}
+// Block-table entry of position `pos` (a ring of mbps entries with a window).
+__device__ __forceinline__ int entry_of(const Params &p, int pos)
+{
+    return p.window > 0 ? (pos / p.bs) % p.mbps : pos / p.bs;
+}
+// Valid rows of the 16-key tile starting at position tb: below the context
+// end and (with a window) at or after its first key.
+__device__ __forceinline__ uint32_t tile_rows(int ctx, int window, int tb)
+{
+    const int nv = min(TT, ctx - tb);
+    const int f = window > 0 ? max(0, ctx - window - tb) : 0;
+    return ((1u << nv) - 1u) & ~((1u << f) - 1u);
+}
 
 // Exclusive prefixes over the B sequences, by one warp: s_pref[i] of the
 // tiles (tiles_of(s_ctx) * Hkv), s_cpref[i] of the cost units (Hkv * (tiles +
 // kCtxCost) for a sequence with tiles). s_pref[B] is the number of tiles,
 // s_cpref[B] the length of the cost space.
-__device__ __forceinline__ void tile_prefix(const int *s_ctx, int *s_pref, int *s_cpref, int B, int Hkv, int lane)
+__device__ __forceinline__ void tile_prefix(const int *s_ctx, int *s_pref, int *s_cpref, int B, int Hkv, int lane,
+                                            int window)
 {
     int run = 0, crun = 0;
     for (int base = 0; base < B; base += 32) {
         const int i = base + lane;
-        const int nt = i < B ? tiles_of(s_ctx[i]) : 0;
+        const int nt = i < B ? tiles_of(s_ctx[i], window) : 0;
         const int v = nt * Hkv, cv = nt > 0 ? (nt + kCtxCost) * Hkv : 0;
         int x = v, cx = cv;
 #pragma unroll
@@ -250,7 +274,7 @@ __device__ __forceinline__ int active_warps(const Params &p, int total)
 // tile whose cost position is at least U (the tiles of context (r, h) sit at
 // cost positions s_cpref[r] + h*(nt + kCtxCost) + kCtxCost + i).
 __device__ __forceinline__ int cost_to_tile(int64_t U, const int *s_ctx, const int *s_pref, const int *s_cpref,
-                                            int B)
+                                            int B, int window)
 {
     if (U >= s_cpref[B]) return s_pref[B];
     int lo = 0, hi = B;  // s_cpref[lo] <= U < s_cpref[hi]
@@ -259,7 +283,7 @@ __device__ __forceinline__ int cost_to_tile(int64_t U, const int *s_ctx, const i
         if (s_cpref[mid] <= U) lo = mid;
         else hi = mid;
     }
-    const int nt = tiles_of(s_ctx[lo]), span = nt + kCtxCost;
+    const int nt = tiles_of(s_ctx[lo], window), span = nt + kCtxCost;
     const int local = static_cast<int>(U - s_cpref[lo]);
     const int h = local / span, off = local - h * span;
     return s_pref[lo] + h * nt + max(0, off - kCtxCost);
@@ -482,7 +506,7 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
         }
     }
     __syncthreads();
-    if (warp == 0) tile_prefix(s_ctx, s_pref, s_cpref, B, Hkv, lane);
+    if (warp == 0) tile_prefix(s_ctx, s_pref, s_cpref, B, Hkv, lane, p.window);
     __syncthreads();
 
     grid_launch_dependents();  // the next grid may be placed (it waits for this one)
@@ -492,8 +516,8 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
     const int W = active_warps(p, total);
     const int w = blockIdx.x * NW + warp;
     if (w >= W) return;
-    const int t_begin = cost_to_tile(static_cast<int64_t>(w) * TC / W, s_ctx, s_pref, s_cpref, B);
-    const int t_end = cost_to_tile(static_cast<int64_t>(w + 1) * TC / W, s_ctx, s_pref, s_cpref, B);
+    const int t_begin = cost_to_tile(static_cast<int64_t>(w) * TC / W, s_ctx, s_pref, s_cpref, B, p.window);
+    const int t_end = cost_to_tile(static_cast<int64_t>(w + 1) * TC / W, s_ctx, s_pref, s_cpref, B, p.window);
     if (t_begin >= t_end) return;  // no CTA-wide barrier follows
 
     // barriers: [warp][stage][K, V] "tile half landed"
@@ -511,7 +535,7 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
         }
         c.t = t;
         c.r = lo;
-        c.nt = tiles_of(s_ctx[lo]);
+        c.nt = tiles_of(s_ctx[lo], p.window);
         const int local = t - s_pref[lo];
         c.h = local / c.nt;
         c.ti = local - c.h * c.nt;
@@ -524,8 +548,8 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
                 c.h = 0;
                 do {
                     ++c.r;
-                } while (c.r < B && tiles_of(s_ctx[c.r]) == 0);
-                if (c.r < B) c.nt = tiles_of(s_ctx[c.r]);
+                } while (c.r < B && tiles_of(s_ctx[c.r], p.window) == 0);
+                if (c.r < B) c.nt = tiles_of(s_ctx[c.r], p.window);
             }
         }
     };
@@ -539,8 +563,8 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
     const uint64_t l2pol = l2_evict_first_policy();
 
     // Copy descriptors of 32 consecutive tiles, one per lane: the element
-    // offset of the tile's K (and V) run in the layer pool and its number of
-    // valid tokens (0: block id outside the pool).
+    // offset of the tile's K (and V) run in the layer pool and its mask of
+    // valid rows (0: block id outside the pool).
     int64_t d_off = 0;
     int d_nv = 0, dbase = 0, d_q = -1;
     auto load_desc = [&](int base) {
@@ -555,12 +579,12 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
             // a segment starts here: its queries are wanted when this tile is
             if (c.ti == 0 || i == 0) d_q = c.r * p.Hq + c.h * G;
             const int ctx = s_ctx[c.r];
-            const int tb = c.ti * TT;
-            const int blk = p.bt[static_cast<size_t>(c.r) * p.mbps + tb / p.bs];
+            const int tb = (first_tile(ctx, p.window) + c.ti) * TT;  // position of the tile's first key
+            const int blk = p.bt[static_cast<size_t>(c.r) * p.mbps + entry_of(p, tb)];
             if (blk >= 0 && blk < p.num_blocks) {
                 d_off = static_cast<int64_t>(blk) * blk_stride + static_cast<int64_t>(c.h) * p.bs * D +
                         static_cast<int64_t>(tb % p.bs) * D;
-                d_nv = min(TT, ctx - tb);
+                d_nv = static_cast<int>(tile_rows(ctx, p.window, tb));
             } else {
                 report(p.status, KVP_ERANGE, c.r);
             }
@@ -571,7 +595,7 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
         Cursor c;
         locate(t_begin + i, c);
         const int ctx = s_ctx[c.r];
-        const int tb = c.ti * TT;
+        const int tb = (first_tile(ctx, p.window) + c.ti) * TT;
         const int32_t *btr = p.bt + static_cast<size_t>(c.r) * p.mbps;
         const uint32_t bar = kbar0 + (st * 2 + half) * 8;
         uint16_t *dst = wst + st * (S::STAGE_BYTES / 2) + half * S::TILE_WORDS;
@@ -579,7 +603,7 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
         uint32_t bytes = 0;
         int nv = 0;
         for (int t = 0; t < TT && tb + t < ctx; t += p.bs) {
-            const int b = btr[(tb + t) / p.bs];
+            const int b = btr[entry_of(p, tb + t)];
             if (b >= 0 && b < p.num_blocks) {
                 bytes += p.bs * D * 2;
                 nv = t + min(p.bs, ctx - tb - t);
@@ -591,14 +615,14 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
         if (bytes) {
             mbar_arrive_expect_tx(bar, bytes);
             for (int t = 0; t < nv; t += p.bs) {
-                const int b = btr[(tb + t) / p.bs];
+                const int b = btr[entry_of(p, tb + t)];
                 bulk_g2s_hint(smem_addr(dst + t * D), src + b * blk_stride + static_cast<size_t>(c.h) * p.bs * D,
                               p.bs * D * 2, bar, l2pol);
             }
         } else {
             mbar_arrive(bar);
         }
-        if (half == 0) nvalid[st] = nv;
+        if (half == 0) nvalid[st] = nv > 0 ? static_cast<int>(tile_rows(ctx, p.window, tb) & ((1u << nv) - 1u)) : 0;
     };
     // Issues half (0: K, 1: V) of tile i (warp-relative) into stage st.
     auto issue = [&](int i, int half, int st) {
@@ -686,8 +710,7 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
             if (lane == 0) report(p.status, KVP_ETIMEOUT, cons.r);
             return;
         }
-        const int nv = nvalid[st];
-        const uint32_t mask = (1u << nv) - 1u;
+        const uint32_t mask = static_cast<uint32_t>(nvalid[st]);  // valid rows of the tile
         const uint16_t *sk = wst + st * (S::STAGE_BYTES / 2) + j * 8;
         const uint16_t *sv = sk + S::TILE_WORDS;
 
@@ -838,7 +861,7 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
             }
         };
         if (mask == 0xFFFFu) tile_qk(std::true_type{});
-        else if (nv > 0) tile_qk(std::false_type{});
+        else if (mask != 0) tile_qk(std::false_type{});
         __syncwarp();  // K half and the previous P are free
         if (seq + NST < ntile) issue(seq + NST, 0, st);
         if (!__all_sync(0xffffffffu, mbar_wait_bounded(kbar0 + st * 16 + 8, par))) {
@@ -846,7 +869,7 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
             return;
         }
         if (mask == 0xFFFFu) tile_pv(std::true_type{});
-        else if (nv > 0) tile_pv(std::false_type{});
+        else if (mask != 0) tile_pv(std::false_type{});
         __syncwarp();  // V half and P buffer are free
         if (seq + NST < ntile) issue(seq + NST, 1, st);
 
@@ -1105,7 +1128,7 @@ __global__ void __launch_bounds__(TcShape<D>::NW * 32, 1)
         }
     }
     __syncthreads();
-    if (warp == 0) tile_prefix(s_ctx, s_pref, s_cpref, B, Hkv, lane);
+    if (warp == 0) tile_prefix(s_ctx, s_pref, s_cpref, B, Hkv, lane, p.window);
     __syncthreads();
     grid_launch_dependents();
 
@@ -1113,8 +1136,8 @@ __global__ void __launch_bounds__(TcShape<D>::NW * 32, 1)
     const int W = active_warps(p, total);
     const int w = blockIdx.x * NW + warp;
     if (w >= W) return;
-    const int t_begin = cost_to_tile(static_cast<int64_t>(w) * TC / W, s_ctx, s_pref, s_cpref, B);
-    const int t_end = cost_to_tile(static_cast<int64_t>(w + 1) * TC / W, s_ctx, s_pref, s_cpref, B);
+    const int t_begin = cost_to_tile(static_cast<int64_t>(w) * TC / W, s_ctx, s_pref, s_cpref, B, p.window);
+    const int t_end = cost_to_tile(static_cast<int64_t>(w + 1) * TC / W, s_ctx, s_pref, s_cpref, B, p.window);
     if (t_begin >= t_end) return;  // no CTA-wide barrier follows
 
     const uint32_t kbar0 = smem_addr(&bars[warp * NST * 2]);
@@ -1131,7 +1154,7 @@ __global__ void __launch_bounds__(TcShape<D>::NW * 32, 1)
         }
         c.t = t;
         c.r = lo;
-        c.nt = tiles_of(s_ctx[lo]);
+        c.nt = tiles_of(s_ctx[lo], p.window);
         const int local = t - s_pref[lo];
         c.h = local / c.nt;
         c.ti = local - c.h * c.nt;
@@ -1144,8 +1167,8 @@ __global__ void __launch_bounds__(TcShape<D>::NW * 32, 1)
                 c.h = 0;
                 do {
                     ++c.r;
-                } while (c.r < B && tiles_of(s_ctx[c.r]) == 0);
-                if (c.r < B) c.nt = tiles_of(s_ctx[c.r]);
+                } while (c.r < B && tiles_of(s_ctx[c.r], p.window) == 0);
+                if (c.r < B) c.nt = tiles_of(s_ctx[c.r], p.window);
             }
         }
     };
@@ -1156,8 +1179,9 @@ __global__ void __launch_bounds__(TcShape<D>::NW * 32, 1)
     const uint64_t l2pol = l2_evict_first_policy();
 
     // copy descriptors of 32 consecutive tiles, one per lane: tensor
-    // coordinates (block * Hkv + head, first row in the block), valid
-    // tokens (0: block id outside the pool) and the segment's query row
+    // coordinates (block * Hkv + head, first row in the block), valid rows
+    // [f, nv) packed as nv | f << 8 (0: block id outside the pool) and the
+    // segment's query row
     int d_tile = 0, d_row = 0, d_nv = 0, d_q = -1, dbase = 0;
     auto load_desc = [&](int base) {
         dbase = base;
@@ -1169,12 +1193,12 @@ __global__ void __launch_bounds__(TcShape<D>::NW * 32, 1)
             locate(t_begin + i, c);
             if (c.ti == 0 || i == 0) d_q = c.r * p.Hq + c.h * G;
             const int ctx = s_ctx[c.r];
-            const int tb = c.ti * TT;
-            const int blk = p.bt[static_cast<size_t>(c.r) * p.mbps + tb / p.bs];
+            const int tb = (first_tile(ctx, p.window) + c.ti) * TT;  // position of the tile's first key
+            const int blk = p.bt[static_cast<size_t>(c.r) * p.mbps + entry_of(p, tb)];
             if (blk >= 0 && blk < p.num_blocks) {
                 d_tile = blk * Hkv + c.h;
                 d_row = tb % p.bs;
-                d_nv = min(TT, ctx - tb);
+                d_nv = min(TT, ctx - tb) | (p.window > 0 ? max(0, ctx - p.window - tb) : 0) << 8;
             } else {
                 report(p.status, KVP_ERANGE, c.r);
             }
@@ -1247,7 +1271,7 @@ __global__ void __launch_bounds__(TcShape<D>::NW * 32, 1)
             if (lane == 0) report(p.status, KVP_ETIMEOUT, cons.r);
             return;
         }
-        const int nv = nvalid[st];
+        const int nv = nvalid[st] & 0xFF, f0 = nvalid[st] >> 8;  // valid rows [f0, nv)
         const uint32_t kt = ring + st * S::STAGE_BYTES, vt = kt + S::HALF_BYTES;
         // ldmatrix row of this lane: matrix lane/8 covers tokens 8*(lane/16) ..
         // and the 8-column chunk (lane/8) % 2 of each 16-column step
@@ -1280,10 +1304,10 @@ __global__ void __launch_bounds__(TcShape<D>::NW * 32, 1)
             // scores of head g at tokens 2q4, 2q4+1, 8+2q4, 9+2q4 (masked by select)
             float x[4] = {sc[0][0], sc[0][1], sc[1][0], sc[1][1]};
             const int t0 = 2 * q4;
-            if (t0 >= nv) x[0] = -INFINITY;
-            if (t0 + 1 >= nv) x[1] = -INFINITY;
-            if (t0 + 8 >= nv) x[2] = -INFINITY;
-            if (t0 + 9 >= nv) x[3] = -INFINITY;
+            if (t0 >= nv || t0 < f0) x[0] = -INFINITY;
+            if (t0 + 1 >= nv || t0 + 1 < f0) x[1] = -INFINITY;
+            if (t0 + 8 >= nv || t0 + 8 < f0) x[2] = -INFINITY;
+            if (t0 + 9 >= nv || t0 + 9 < f0) x[3] = -INFINITY;
             float mt = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
             mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
             mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
@@ -1316,12 +1340,17 @@ __global__ void __launch_bounds__(TcShape<D>::NW * 32, 1)
                 const float2 h1 = unpack2<BF16>(ph1), l1 = unpack2<BF16>(pl1);
                 l_run += ((h0.x + l0.x) + (h0.y + l0.y)) + ((h1.x + l1.x) + (h1.y + l1.y));
             }
-            if (nv < TT) {
+            if (nv < TT || f0 > 0) {
                 // V rows past the context may hold anything (never-written
-                // slots): zero them so 0 * V stays 0 in the product
+                // slots), and so may rows before a window: zero them so
+                // 0 * V stays 0 in the product
                 const uint4 z = make_uint4(0u, 0u, 0u, 0u);
                 for (int k = lane; k < (TT - nv) * (D / 8); k += 32) {
                     const int row = nv + k / (D / 8), c8 = k % (D / 8);
+                    *reinterpret_cast<uint4 *>(smem + (tc_addr<D>(vt, row, c8) - smem_addr(smem))) = z;
+                }
+                for (int k = lane; k < f0 * (D / 8); k += 32) {
+                    const int row = k / (D / 8), c8 = k % (D / 8);
                     *reinterpret_cast<uint4 *>(smem + (tc_addr<D>(vt, row, c8) - smem_addr(smem))) = z;
                 }
                 __syncwarp();
@@ -1448,7 +1477,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const Param
         s_ctx[i] = ctx_ok(p, c) ? c : -1;
     }
     __syncthreads();
-    if (warp == 0) tile_prefix(s_ctx, s_pref, s_cpref, B, Hkv, lane);
+    if (warp == 0) tile_prefix(s_ctx, s_pref, s_cpref, B, Hkv, lane, p.window);
     __syncthreads();
     const int total = s_pref[B], TC = s_cpref[B];
     const int W = active_warps(p, total);
@@ -1460,7 +1489,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const Param
     for (int task = blockIdx.x * kCombineWarps + warp; task < ntask; task += gridDim.x * kCombineWarps) {
         const int g = task % G, rh = task / G;
         const int r = rh / Hkv, h = rh - r * Hkv;
-        const int nt = tiles_of(s_ctx[r]);
+        const int nt = tiles_of(s_ctx[r], p.window);
         if (nt == 0) continue;
         int w_first, w_last;
         context_warps(s_cpref[r] + h * (nt + kCtxCost) + kCtxCost, nt, W, TC, w_first, w_last);
@@ -1679,6 +1708,9 @@ extern "C" int paged_decode_attention(kvp_pool *pool, int layer, const kvp_attn_
     if ((rc = resolve_attn(pool, attn, &Hq, &Hkv, &G))) return rc;
     if (B == 0) return KVP_OK;
     if (max_blocks_per_seq <= 0) return set_error(KVP_EINVAL, "max_blocks_per_seq must be > 0");
+    if (attn->window > 0 && static_cast<int64_t>(max_blocks_per_seq) * pool->cfg.block_size < attn->window)
+        return set_error(KVP_EINVAL, "a ring of %d blocks of %d cannot hold the window of %d", max_blocks_per_seq,
+                         pool->cfg.block_size, attn->window);
     if (!q || !block_tables || !ctx_lens || !out || !workspace)
         return set_error(KVP_EINVAL, "paged_decode_attention: a required pointer is NULL");
     if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(out)) & 15)
@@ -1698,6 +1730,7 @@ extern "C" int paged_decode_attention(kvp_pool *pool, int layer, const kvp_attn_
     p.B = B, p.Hq = Hq, p.Hkv = Hkv, p.mbps = max_blocks_per_seq, p.bs = pool->cfg.block_size;
     p.num_blocks = pool->cfg.num_blocks, p.max_ctx = max_ctx_len, p.max_seq_len = pool->cfg.max_seq_len;
     p.warps_total = L.warps_total, p.min_tiles = L.min_tiles;
+    p.window = attn->window;
     const double scale = static_cast<double>(static_cast<float>(1.0 / sqrt(static_cast<double>(pool->cfg.head_dim))));
     p.qscale = static_cast<float>(scale * 1.4426950408889634);  // log2(e): softmax via exp2
     const bool bf16 = pool->cfg.kv_dtype == KVP_BF16;

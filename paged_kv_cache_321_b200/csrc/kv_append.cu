@@ -1,5 +1,5 @@
-// kv_append: per-head q/k RMSNorm -> rotate-half RoPE -> fp32 -> fp16/bf16
-// (nearest, ties to even) -> scatter into the token's block slot.
+// kv_append: per-head q/k RMSNorm -> RoPE -> fp32 -> fp16/bf16 (nearest,
+// ties to even) -> scatter into the token's block slot.
 //
 // The step of makarna/pkg/model/arch/hybrid_decoder.go (runHybridAttentionBlock:
 // QNorm/KNorm, RoPE, cache.Append) fused into one launch, with the slot rule
@@ -10,7 +10,10 @@
 //
 // Mapping: one warp per (token, row), rows = Hq query heads, Hkv key heads,
 // Hkv value heads. Lane l owns the D/32 consecutive elements starting at
-// l*D/32, so for rotate-half the partner of every element sits in lane l^16.
+// l*D/32, so for full rotate-half RoPE the partner of every element sits in
+// lane l^16; partial or interleaved RoPE (the per-layer rope_dim of
+// forward_layer in soft3/glia/run/arch/decoder/forward.rs) reads the partner
+// from the row staged in shared memory.
 // The sum of squares is taken in order d = 0..D-1 from shared memory (every
 // lane reads the same addresses, a broadcast), each product and sum a
 // separate IEEE operation; RoPE uses separately rounded products and sums.
@@ -29,6 +32,7 @@ struct AppendParams {
     float *q_out;
     int *status;
     int T, S, Hq, Hkv, bs, mbps, num_blocks, max_seq_len, rope_max_pos;
+    int R, style, window;  // rotary width, pairing, sliding window (> 0: ring rows)
     float eps;
 };
 
@@ -133,7 +137,7 @@ __global__ void __launch_bounds__(kAppendWarps * 32) kv_append_kernel(const Appe
 #pragma unroll
             for (int e = 0; e < E; ++e) x.x[e] = __fmul_rn(__fmul_rn(x.x[e], inv), wv.x[e]);
         }
-        if (p.rope != nullptr) {
+        if (p.rope != nullptr && p.R == D && p.style == KVP_ROPE_HALF) {
             // lanes 0..15 hold dims [0, D/2), lanes 16..31 the partners [D/2, D)
             const float2 *cs = p.rope + static_cast<int64_t>(pos) * (D / 2) + (lane & 15) * E;
             const bool lower = lane < 16;
@@ -144,6 +148,27 @@ __global__ void __launch_bounds__(kAppendWarps * 32) kv_append_kernel(const Appe
                 x.x[e] = lower ? __fsub_rn(__fmul_rn(x.x[e], c.x), __fmul_rn(other, c.y))
                                : __fadd_rn(__fmul_rn(x.x[e], c.x), __fmul_rn(other, c.y));
             }
+        } else if (p.rope != nullptr) {
+            // pair i turns (a, b) = (i, i + R/2) or (2i, 2i + 1) of the first
+            // R dims: y_a = x_a c - x_b s, y_b = x_b c + x_a s
+            __syncwarp();  // every lane is done reading the norm's staging
+            x.store(&rowbuf[wib][lane * E]);
+            __syncwarp();
+            const float2 *cs = p.rope + static_cast<int64_t>(pos) * (p.R / 2);
+            const int hr = p.R / 2;
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const int d = lane * E + e;
+                if (d >= p.R) continue;
+                const bool inter = p.style == KVP_ROPE_INTERLEAVED;
+                const bool lower = inter ? (d & 1) == 0 : d < hr;
+                const int i = inter ? d >> 1 : (lower ? d : d - hr);
+                const int partner = inter ? d ^ 1 : (lower ? d + hr : d - hr);
+                const float other = rowbuf[wib][partner];
+                const float2 c = cs[i];
+                x.x[e] = lower ? __fsub_rn(__fmul_rn(x.x[e], c.x), __fmul_rn(other, c.y))
+                               : __fadd_rn(__fmul_rn(x.x[e], c.x), __fmul_rn(other, c.y));
+            }
         }
         if (kind == 0) {
             x.store(p.q_out + (static_cast<int64_t>(t) * p.Hq + head) * D + lane * E);
@@ -151,8 +176,9 @@ __global__ void __launch_bounds__(kAppendWarps * 32) kv_append_kernel(const Appe
         }
     }
 
-    // K or V row: resolve the slot (GetBlockForPosition / GetBlockOffset)
-    const int j = pos / p.bs, slot = pos % p.bs;
+    // K or V row: resolve the slot (GetBlockForPosition / GetBlockOffset);
+    // with a sliding window the row is a ring of mbps entries
+    const int j = p.window > 0 ? (pos / p.bs) % p.mbps : pos / p.bs, slot = pos % p.bs;
     if (j >= p.mbps) {
         if (lane == 0) report(p.status, KVP_ERANGE, t);
         return;
@@ -197,6 +223,9 @@ extern "C" int kv_append(kvp_pool *pool, int layer, const kvp_attn_config *attn,
         return set_error(KVP_EINVAL, "kv_append: a required pointer is NULL");
     if (rope_table && rope_max_pos <= 0) return set_error(KVP_EINVAL, "rope_max_pos must be > 0");
     const int D = pool->cfg.head_dim;
+    if (attn->window > 0 && static_cast<int64_t>(max_blocks_per_seq) * pool->cfg.block_size < attn->window)
+        return set_error(KVP_EINVAL, "a ring of %d blocks of %d cannot hold the window of %d", max_blocks_per_seq,
+                         pool->cfg.block_size, attn->window);
     const uintptr_t align = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
                             reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(q_out) |
                             reinterpret_cast<uintptr_t>(q_norm_w) | reinterpret_cast<uintptr_t>(k_norm_w) |
@@ -212,6 +241,7 @@ extern "C" int kv_append(kvp_pool *pool, int layer, const kvp_attn_config *attn,
     p.T = T, p.S = num_seqs, p.Hq = Hq, p.Hkv = Hkv, p.bs = pool->cfg.block_size, p.mbps = max_blocks_per_seq;
     p.num_blocks = pool->cfg.num_blocks, p.max_seq_len = pool->cfg.max_seq_len;
     p.rope_max_pos = rope_table ? rope_max_pos : 0;
+    p.R = attn->rope_dim == 0 ? D : attn->rope_dim, p.style = attn->rope_style, p.window = attn->window;
     p.eps = attn->rms_eps;
     const bool bf16 = pool->cfg.kv_dtype == KVP_BF16;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -53,6 +53,12 @@ int resolve_attn(const kvp_pool *pool, const kvp_attn_config *attn, int *Hq, int
         return set_error(KVP_EINVAL, "head_dim %d differs from the pool's %d", attn->head_dim, pool->cfg.head_dim);
     if (hkv != pool->cfg.num_kv_heads)
         return set_error(KVP_EINVAL, "num_kv_heads %d differs from the pool's %d", hkv, pool->cfg.num_kv_heads);
+    if (attn->rope_dim < 0 || attn->rope_dim > attn->head_dim || (attn->rope_dim & 1))
+        return set_error(KVP_EINVAL, "rope_dim %d must be 0 or even and <= head_dim", attn->rope_dim);
+    if (attn->rope_style != KVP_ROPE_HALF && attn->rope_style != KVP_ROPE_INTERLEAVED)
+        return set_error(KVP_EINVAL, "rope_style %d is neither KVP_ROPE_HALF nor KVP_ROPE_INTERLEAVED",
+                         attn->rope_style);
+    if (attn->window < 0) return set_error(KVP_EINVAL, "window %d must be >= 0", attn->window);
     *Hq = hq;
     *Hkv = hkv;
     *G = hq / hkv;
@@ -170,10 +176,17 @@ int kv_pool_sync_status(kvp_pool *pool, void *stream, int *device_code)
     return set_error(KVP_EDEVICE, "device error %d (%s), detail %d", st[0], what, st[1]);
 }
 
+// Rotary width of a config: rope_dim, or head_dim when 0 (-1 if invalid).
+static int rotary_width(const kvp_attn_config *attn)
+{
+    const int D = attn->head_dim, R = attn->rope_dim == 0 ? D : attn->rope_dim;
+    return (D <= 0 || (D & 1) || R <= 0 || R > D || (R & 1)) ? -1 : R;
+}
+
 size_t kvp_rope_table_bytes(const kvp_attn_config *attn, int max_pos)
 {
-    if (!attn || attn->head_dim <= 0 || (attn->head_dim & 1) || max_pos <= 0) return 0;
-    return static_cast<size_t>(max_pos) * attn->head_dim * sizeof(float);
+    if (!attn || rotary_width(attn) < 0 || max_pos <= 0) return 0;
+    return static_cast<size_t>(max_pos) * rotary_width(attn) * sizeof(float);
 }
 
 int kvp_rope_table_fill(const kvp_attn_config *attn, int max_pos, float *table)
@@ -182,15 +195,17 @@ int kvp_rope_table_fill(const kvp_attn_config *attn, int max_pos, float *table)
     const int D = attn->head_dim;
     if (D <= 0 || D > 256 || (D & 1))
         return set_error(KVP_EUNSUPPORTED, "rope needs an even head_dim <= 256 (got %d)", D);
+    const int R = rotary_width(attn);
+    if (R < 0) return set_error(KVP_EINVAL, "rope_dim %d must be 0 or even and <= head_dim", attn->rope_dim);
     if (!(attn->rope_theta > 0.0f)) return set_error(KVP_EINVAL, "rope_theta must be > 0");
     if (max_pos <= 0) return set_error(KVP_EINVAL, "max_pos must be > 0");
-    const int half = D / 2;
+    const int half = R / 2;
     const double theta = static_cast<double>(attn->rope_theta);
     std::vector<double> inv_freq(half);
-    for (int i = 0; i < half; ++i) inv_freq[i] = ::pow(theta, -(2.0 * static_cast<double>(i)) / static_cast<double>(D));
-    std::vector<float> host(static_cast<size_t>(max_pos) * D);
+    for (int i = 0; i < half; ++i) inv_freq[i] = ::pow(theta, -(2.0 * static_cast<double>(i)) / static_cast<double>(R));
+    std::vector<float> host(static_cast<size_t>(max_pos) * R);
     for (int p = 0; p < max_pos; ++p) {
-        float *row = host.data() + static_cast<size_t>(p) * D;
+        float *row = host.data() + static_cast<size_t>(p) * R;
         for (int i = 0; i < half; ++i) {
             const double ang = static_cast<double>(p) * inv_freq[i];
             row[2 * i] = static_cast<float>(::cos(ang));

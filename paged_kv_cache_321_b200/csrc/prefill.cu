@@ -34,6 +34,7 @@
 //  * the epilogue reads O from TMEM, divides by the row sum and writes fp32.
 #include <cuda.h>
 
+#include <climits>
 #include <math.h>
 
 #include "common.cuh"
@@ -87,8 +88,28 @@ struct Params {
     int *status;
     int S, Hq, Hkv, G, mbps, bs, num_blocks, max_seq_len, ntq;  // ntq: query tiles per sequence (grid)
     int nbins;              // cost bins: KV tiles an item can read, 0 .. max_seq_len / BN + 1
+    int window;             // sliding window in keys (0: none); > 0 makes block-table rows rings
     float qscale;           // softmax scale * log2(e), folded into Q
 };
+
+// A sequence the kernel refuses: an empty or over-long chunk, a context past
+// the table (without a window) or max_seq_len, or (with a ring) a chunk whose
+// own later keys have overwritten a ring slot one of its queries still needs
+// (the smallest key needed, max(0, first query position - window + 1), must
+// be newer than ctx - 1 - mbps * bs).
+__device__ __forceinline__ bool seq_refused(const Params &p, int q_len, int ctx)
+{
+    if (q_len <= 0 || ctx < q_len || ctx > p.max_seq_len) return true;
+    if (p.window == 0) return ctx > p.mbps * p.bs;
+    const int need = max(0, ctx - q_len - p.window + 1);
+    return static_cast<int64_t>(need) + static_cast<int64_t>(p.mbps) * p.bs <= ctx - 1;
+}
+
+// First KV tile (of BN keys) the query at position `pos` needs.
+__device__ __forceinline__ int first_kv_tile(const Params &p, int pos)
+{
+    return p.window > 0 ? max(0, pos - p.window + 1) / BN : 0;
+}
 
 // ---------------------------------------------------------------- PTX
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int c0, int c1, int c2, uint32_t bar)
@@ -238,8 +259,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         auto cost = [&](int i) -> int {
             const int si = i / p.ntq, t0i = (i - si * p.ntq) * TQ;
             const int ql = p.cu_q[si + 1] - p.cu_q[si], c = p.ctx[si];
-            if (t0i >= ql || ql <= 0 || c < ql || c > p.mbps * p.bs || c > p.max_seq_len) return 0;
-            return (c - ql + min(ql, t0i + TQ) - 1) / BN + 1;
+            if (t0i >= ql || seq_refused(p, ql, c)) return 0;
+            return (c - ql + min(ql, t0i + TQ) - 1) / BN + 1 - first_kv_tile(p, c - ql + t0i);
         };
         for (int i = tid; i < p.nbins; i += NTHREADS) hist[i] = 0;
         __syncthreads();
@@ -294,8 +315,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int ctx = p.ctx[s];
     const int t0 = qt * TQ;  // first query token of this tile (within the sequence)
     if (t0 >= q_len) return;
-    const bool bad = q_len <= 0 || ctx < q_len || ctx > p.mbps * p.bs || ctx > p.max_seq_len;
-    if (bad) {
+    if (seq_refused(p, q_len, ctx)) {
         if (qt == 0 && h == 0 && tid == 0) report(p.status, KVP_ERANGE, s);
         return;  // uniform for the CTA: nothing allocated yet
     }
@@ -305,7 +325,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     const int first_pos = ctx - q_len;                   // position of query 0
     const int last_pos = first_pos + min(q_len, t0 + TQ) - 1;
-    const int nkv = last_pos / BN + 1;                   // KV tiles this CTA reads
+    const int j0 = first_kv_tile(p, first_pos + t0);     // KV tiles j0 .. j0 + nkv - 1 of the position axis
+    const int nkv = last_pos / BN + 1 - j0;              // KV tiles this CTA reads
 
     if (tid == 0) {
         for (int i = 0; i < NBARS; ++i) {
@@ -339,15 +360,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int kv = warp == V_WARP;
         const int32_t *btr = p.bt + static_cast<size_t>(s) * p.mbps;
         const uint32_t half_rows_bytes = p.bs * 128;  // one block's rows of one 64-column half
-        auto block_of = [&](int j) {
+        auto block_of = [&](int j) {  // j: tile of the position axis
             const int first = (j * BN) / p.bs;
             const int nblk = (min(BN, ctx - j * BN) + p.bs - 1) / p.bs;
-            return lane < nblk ? btr[first + lane] : -1;
+            const int e = p.window > 0 ? (first + lane) % p.mbps : first + lane;  // the ring
+            return lane < nblk ? btr[e] : -1;
         };
-        int blk = block_of(0);
+        int blk = block_of(j0);
         for (int j = 0; j < nkv && !timed_out; ++j) {
             const int st = j % NSTAGE;
-            const int nblk = (min(BN, ctx - j * BN) + p.bs - 1) / p.bs;
+            const int nblk = (min(BN, ctx - (j0 + j) * BN) + p.bs - 1) / p.bs;
             const bool mine = lane < nblk;
             const bool valid = mine && blk >= 0 && blk < p.num_blocks;
             if (mine && !valid && !kv) report(p.status, KVP_ERANGE, s);
@@ -373,7 +395,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 for (int hf = 0; hf < 2; ++hf)
                     tma_load_3d(dst0 + hf * HALF_BYTES, kv ? &tmap_v : &tmap_k, hf * 64, 0, tile, full);
             }
-            if (j + 1 < nkv) blk = block_of(j + 1);
+            if (j + 1 < nkv) blk = block_of(j0 + j + 1);
         }
     } else if (warp == MMA_WARP) {
         // ------------------------------------------------------ MMA issuer
@@ -428,7 +450,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int g = r / TQ, t = r % TQ;
         const int qi = t0 + t;  // query index in the sequence
         const bool row_ok = qi < q_len;
-        const int pos = row_ok ? first_pos + qi : -1;  // sees keys 0..pos
+        const int pos = row_ok ? first_pos + qi : -1;  // sees keys 0..pos (or lo_key..pos)
+        const int lo_key = p.window > 0 ? pos - p.window + 1 : INT_MIN;
         const size_t qrow = (static_cast<size_t>(q0 + qi) * p.Hq + static_cast<size_t>(h) * G + g) * D;
         float *xch = reinterpret_cast<float *>(smem + XCH_OFF);  // [parity][half][row]
         // publishes v for this row and returns the partner half's value for
@@ -483,17 +506,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_SFREE + b));
-            // causal mask (skipped when all 64 keys are visible to every row
-            // of the warp, as for all but the diagonal tiles) and row max
-            const int key0 = j * BN + col0;
+            // causal (and window) mask, skipped when all 64 keys are visible
+            // to every row of the warp, as for all but the diagonal tiles
+            // (and the window's edge), and row max
+            const int key0 = (j0 + j) * BN + col0;
             float mx = -INFINITY;
-            if (__all_sync(0xffffffffu, key0 + 63 <= pos)) {
+            if (__all_sync(0xffffffffu, key0 + 63 <= pos && key0 >= lo_key)) {
 #pragma unroll
                 for (int i = 0; i < 64; ++i) mx = fmaxf(mx, sv[i]);
             } else {
 #pragma unroll
                 for (int i = 0; i < 64; ++i) {
-                    if (key0 + i > pos) sv[i] = -INFINITY;
+                    if (key0 + i > pos || key0 + i < lo_key) sv[i] = -INFINITY;
                     mx = fmaxf(mx, sv[i]);
                 }
             }
@@ -533,6 +557,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 l *= alpha;
             }
             if (move) m_ref = mx;
+            // With a window a row may see no key of a tile (m_ref still -inf):
+            // its scores are all -inf, and a finite reference keeps P at 0
+            const float mr = (p.window > 0 && m_ref == -INFINITY) ? 0.0f : m_ref;
             // P = exp2(s - m_ref) rounded to 16 bits; l sums the rounded values
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
@@ -540,11 +567,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float x0 = sv[c * 8 + 2 * e], x1 = sv[c * 8 + 2 * e + 1];
-                    // a masked score gives exp2(-inf) = 0; m_ref is finite from
-                    // the first tile on in every row that has a query (key 0 is
-                    // visible to all), rows past the chunk are never stored
-                    const float p0 = ex2(x0 - m_ref);
-                    const float p1 = ex2(x1 - m_ref);
+                    // a masked score gives exp2(-inf) = 0: without a window m_ref
+                    // is finite from the first tile on in every row that has a
+                    // query (key 0 is visible to all), with one mr is; rows past
+                    // the chunk are never stored
+                    const float p0 = ex2(x0 - mr);
+                    const float p1 = ex2(x1 - mr);
                     w[e] = pack2<BF16>(p0, p1);
                     const float2 back = unpack<BF16>(w[e]);
                     l += back.x + back.y;
@@ -554,7 +582,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             // keys of this tile past the context: their V rows may hold
             // anything (or were not loaded); zero them so 0 * V stays 0
-            const int nkeys = min(BN, ctx - j * BN);
+            const int nkeys = min(BN, ctx - (j0 + j) * BN);
             if (nkeys < BN) {
                 const int st = j % NSTAGE;
                 if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar(B_VFULL + st), (j / NSTAGE) & 1))) {
@@ -661,6 +689,10 @@ extern "C" int paged_prefill_attention(kvp_pool *pool, int layer, const kvp_attn
     p.S = S, p.Hq = Hq, p.Hkv = Hkv, p.G = G, p.mbps = max_blocks_per_seq, p.bs = bs;
     p.num_blocks = pool->cfg.num_blocks, p.max_seq_len = pool->cfg.max_seq_len;
     p.nbins = pool->cfg.max_seq_len / pre::BN + 2;
+    p.window = attn->window;
+    if (attn->window > 0 && static_cast<int64_t>(max_blocks_per_seq) * bs < attn->window)
+        return set_error(KVP_EINVAL, "a ring of %d blocks of %d cannot hold the window of %d", max_blocks_per_seq, bs,
+                         attn->window);
     const double scale = static_cast<double>(static_cast<float>(1.0 / sqrt(static_cast<double>(pre::D))));
     p.qscale = static_cast<float>(scale * 1.4426950408889634);
     const bool bf16 = pool->cfg.kv_dtype == KVP_BF16;

@@ -24,7 +24,8 @@ class GpuRun:
                            device=dev)
         self.pool.k.copy_(torch.from_numpy(wl.pool_k.view(np.int16)))
         self.pool.v.copy_(torch.from_numpy(wl.pool_v.view(np.int16)))
-        self.attn = K.attn_config(sp.Hq, sp.Hkv, sp.D, float(np.float32(sp.theta)), sp.eps)
+        self.attn = K.attn_config(sp.Hq, sp.Hkv, sp.D, float(np.float32(sp.theta)), sp.eps, sp.rope_dim,
+                                  sp.rope_style, sp.window)
         t = lambda a, dt=None: None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(dev)
         self.q, self.k, self.v = t(wl.q), t(wl.k), t(wl.v)
         self.qn, self.kn = t(wl.q_norm_w), t(wl.k_norm_w)
@@ -34,7 +35,7 @@ class GpuRun:
         self.q_out = torch.zeros((wl.T, sp.Hq * sp.D), dtype=torch.float32, device=dev)
         self.rope = None
         if sp.theta:
-            self.rope = torch.empty(wl.max_seq_len * sp.D, dtype=torch.float32, device=dev)
+            self.rope = torch.empty(wl.max_seq_len * (sp.rope_dim or sp.D), dtype=torch.float32, device=dev)
             K.rope_table_fill(self.attn, wl.max_seq_len, self.rope)
 
     def append(self):

@@ -78,3 +78,22 @@ def test_prefill_full_size_sampled(orc):
     st, ref = oracle_rows(orc, wl, q_ref, pk, pv, rows[pick])
     assert st == 0
     assert_close(out.cpu().numpy()[pick], ref, "mixed-prefill sampled rows")
+
+
+def test_prefill_bf16_pool_within_its_bound(orc):
+    # With a bf16 pool the tensor-core operands are bf16 (A and B of one MMA
+    # share a type): q and the softmax weights are rounded to 8 significant
+    # bits (relative error up to 2^-8) instead of fp16's 11, so the error is
+    # about 8x fp16's and the 1e-3 bar does not hold; this pins the bound that
+    # does, 1e-2 + 1e-2*|oracle| (about 2x the largest error seen).
+    wl = make_workload(spec("bf16-pool", kv_dtype="bf16", Hq=16, Hkv=2, bs=32,
+                            segments=(Segment(q_len=150, fixed=(10, 1000)),), seed_offset=207))
+    run = GpuRun(wl, torch.device("cuda", 0))
+    run.append()
+    out, rows = run.prefill()
+    run.pool.sync_status()
+    st, q_ref, pk, pv = orc.workload_append(wl)
+    st, ref = oracle_rows(orc, wl, q_ref, pk, pv, rows)
+    g = out.cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(g))
+    assert np.all(np.abs(g - ref) <= 1e-2 + 1e-2 * np.abs(ref))
