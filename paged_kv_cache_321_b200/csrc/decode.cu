@@ -1304,10 +1304,16 @@ __global__ void __launch_bounds__(TcShape<D>::NW * 32, 1)
             // scores of head g at tokens 2q4, 2q4+1, 8+2q4, 9+2q4 (masked by select)
             float x[4] = {sc[0][0], sc[0][1], sc[1][0], sc[1][1]};
             const int t0 = 2 * q4;
-            if (t0 >= nv || t0 < f0) x[0] = -INFINITY;
-            if (t0 + 1 >= nv || t0 + 1 < f0) x[1] = -INFINITY;
-            if (t0 + 8 >= nv || t0 + 8 < f0) x[2] = -INFINITY;
-            if (t0 + 9 >= nv || t0 + 9 < f0) x[3] = -INFINITY;
+            if (t0 >= nv) x[0] = -INFINITY;
+            if (t0 + 1 >= nv) x[1] = -INFINITY;
+            if (t0 + 8 >= nv) x[2] = -INFINITY;
+            if (t0 + 9 >= nv) x[3] = -INFINITY;
+            if (f0 > 0) {  // a window's first tile: rows before its first key (uniform branch)
+                if (t0 < f0) x[0] = -INFINITY;
+                if (t0 + 1 < f0) x[1] = -INFINITY;
+                if (t0 + 8 < f0) x[2] = -INFINITY;
+                if (t0 + 9 < f0) x[3] = -INFINITY;
+            }
             float mt = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
             mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
             mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
