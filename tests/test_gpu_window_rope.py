@@ -211,3 +211,19 @@ def test_ring_shorter_than_window_refused_on_host():
         K.paged_decode_attention(pool, 0, attn, q, bt, ctx, 1, torch.empty_like(q), ws)
     assert e.value.code == K.KVP_EINVAL
     pool.close()
+
+
+@pytest.mark.parametrize("kw", [dict(rope_dim=33), dict(rope_dim=130), dict(rope_dim=-2), dict(rope_style=2),
+                                dict(window=-1)])
+def test_bad_rope_or_window_fields_refused_on_host(kw):
+    dev = torch.device("cuda", 0)
+    pool = K.Pool(1, 2, 128, 16, 256, 8, "f16", device=dev)
+    attn = K.attn_config(4, 2, 128, 1e4, 1e-6, **kw)
+    T = 1
+    f = lambda n: torch.zeros((T, n), dtype=torch.float32, device=dev)
+    i = torch.zeros(T, dtype=torch.int32, device=dev)
+    bt = torch.zeros((1, 4), dtype=torch.int32, device=dev)
+    with pytest.raises(K.KvpError) as e:
+        K.kv_append(pool, 0, attn, f(4 * 128), f(2 * 128), f(2 * 128), i, i, bt, f(4 * 128))
+    assert e.value.code == K.KVP_EINVAL
+    pool.close()

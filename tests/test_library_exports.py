@@ -54,3 +54,29 @@ def test_host_side_errors_need_no_gpu():
     cfg = K.AttnConfig(32, 8, 128, 5e5, 1e-6)
     assert lib.kvp_rope_table_bytes(ctypes.byref(cfg), 100) == 100 * 128 * 4
     assert lib.kvp_rope_table_fill(ctypes.byref(K.AttnConfig(32, 8, 127, 5e5, 1e-6)), 10, None) != 0
+
+
+def test_rope_table_size_follows_the_rotary_width():
+    # the table holds rope_dim/2 (cos, sin) pairs per position; invalid
+    # widths (odd, wider than the head) size to 0
+    import paged_kv_cache_321_b200 as K
+
+    lib = K.lib()
+    size = lambda **kw: lib.kvp_rope_table_bytes(ctypes.byref(K.attn_config(32, 8, 128, 1e4, 1e-6, **kw)), 100)
+    assert size() == 100 * 128 * 4
+    assert size(rope_dim=32) == 100 * 32 * 4
+    assert size(rope_dim=64, rope_style=K.KVP_ROPE_INTERLEAVED) == 100 * 64 * 4
+    assert size(rope_dim=33) == 0 and size(rope_dim=130) == 0
+    assert lib.kvp_rope_table_fill(ctypes.byref(K.attn_config(32, 8, 128, 1e4, 1e-6, rope_dim=31)), 10, None) != 0
+
+
+def test_attn_config_layout_matches_the_header():
+    # eight 4-byte fields in the header's order; zero-filled extras mean
+    # full rotate-half RoPE and no window
+    import paged_kv_cache_321_b200 as K
+
+    c = K.attn_config(32, 8, 128, 5e5, 1e-6)
+    assert ctypes.sizeof(c) == 32
+    assert (c.rope_dim, c.rope_style, c.window) == (0, K.KVP_ROPE_HALF, 0)
+    assert [f[0] for f in K.AttnConfig._fields_] == ["num_heads", "num_kv_heads", "head_dim", "rope_theta",
+                                                      "rms_eps", "rope_dim", "rope_style", "window"]
