@@ -396,6 +396,25 @@ int kvp_seq_num_blocks(const kvp_seq *seq);
  * too small. */
 int kvp_seq_block_table(const kvp_seq *seq, int layer, int32_t *out, int max_blocks, uint8_t *owned);
 
+/* The entries of layer `layer`'s block-table row that changed since this
+ * sequence's previous call for that layer, for a caller that keeps the row in
+ * device memory and uploads only what changed (the rule of
+ * LayerDevicePtrTables in makarna/pkg/kvcache/paged_cache.go: a layer's
+ * device tables are rebuilt only when its number of blocks grows). Blocks
+ * only ever grow at the end of a row, except when they are replaced
+ * (kvp_seq_allocate_for_tokens, kvp_seq_free). So:
+ *   - first call for the layer, or blocks replaced since the last one: writes
+ *     the whole row (entries past the blocks = -1); *first = 0,
+ *     *end = max_blocks;
+ *   - blocks grew: writes only the new entries; [*first, *end) is their range;
+ *   - otherwise: writes nothing; *first = *end = 0.
+ * `row` is the caller's host copy of the row (max_blocks int32), the same
+ * buffer on every call; entries outside [*first, *end) are left as they are,
+ * so after the call the copy equals kvp_seq_block_table's row.
+ * Errors: KVP_EINVAL for bad arguments; KVP_ERANGE when the sequence holds
+ * more than max_blocks blocks (nothing written, the state unchanged). */
+int kvp_seq_block_table_delta(kvp_seq *seq, int layer, int32_t *row, int max_blocks, int *first, int *end);
+
 #ifdef __cplusplus
 }
 #endif

@@ -116,6 +116,8 @@ class SeqModel:
 
     def __init__(self, pool: PoolModel):
         self.pool = pool
+        self.epoch = 0
+        self.synced = {}  # layer -> (epoch, entries) of the last table delta
         self.free_all()
 
     def free_all(self):
@@ -127,6 +129,23 @@ class SeqModel:
         self.owned = [[] for _ in range(self.pool.num_layers)]
         self.tokens, self.hashes = [], []
         self.computed = self.written = 0
+        self.epoch = getattr(self, "epoch", 0) + 1
+
+    # LayerDevicePtrTables' rule: device rows change only when the number of
+    # blocks grows, or when the sequence's blocks are replaced
+    def table_delta(self, layer, max_blocks):
+        n = len(self.ids[layer])
+        if n > max_blocks:
+            return None
+        ep, done = self.synced.get(layer, (None, 0))
+        if ep != self.epoch:
+            rng = (0, max_blocks)
+        elif n > done:
+            rng = (done, n)
+        else:
+            rng = (0, 0)
+        self.synced[layer] = (self.epoch, n)
+        return rng
 
     def _ensure(self, required):
         p = self.pool

@@ -33,6 +33,7 @@ EXPORTS = (
     "kvp_blocks_create", "kvp_blocks_destroy", "kvp_blocks_count", "kvp_blocks_refs", "kvp_block_hash",
     "kvp_seq_create", "kvp_seq_destroy", "kvp_seq_free", "kvp_seq_allocate_for_tokens", "kvp_seq_append_token",
     "kvp_seq_reserve", "kvp_seq_commit", "kvp_seq_len", "kvp_seq_num_blocks", "kvp_seq_block_table",
+    "kvp_seq_block_table_delta",
 )
 
 
@@ -101,6 +102,7 @@ def lib() -> C.CDLL:
             "kvp_seq_len": (i32, [P]),
             "kvp_seq_num_blocks": (i32, [P]),
             "kvp_seq_block_table": (i32, [P, i32, P, i32, P]),
+            "kvp_seq_block_table_delta": (i32, [P, i32, P, i32, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -334,6 +336,33 @@ class Sequence:
         if rc < 0:
             _check(rc)
         return list(ids)[:n], [bool(x) for x in list(owned)[:n]]
+
+    def block_table_delta(self, layer: int, row) -> tuple:
+        """Updates `row` (a host int32 numpy array, the same one every call)
+        with the entries that changed since the last call for this layer and
+        returns their range (first, end); first == end: nothing changed."""
+        import numpy as np
+
+        assert isinstance(row, np.ndarray) and row.dtype == np.int32 and row.flags.c_contiguous
+        first, end = C.c_int(), C.c_int()
+        _check(lib().kvp_seq_block_table_delta(self.handle, layer, row.ctypes.data_as(C.c_void_p), row.size,
+                                               C.byref(first), C.byref(end)))
+        return first.value, end.value
+
+    def sync_block_table(self, layer: int, row, device_row: torch.Tensor, stream=None) -> tuple:
+        """Keeps a device-resident row equal to the layer's block table,
+        uploading only the entries that changed (growth: the new ones; a
+        replaced prompt: the whole row). `row` is this row's host copy.
+        Returns the uploaded range."""
+        first, end = self.block_table_delta(layer, row)
+        if end > first:
+            src = torch.from_numpy(row[first:end])
+            if stream is not None:
+                with torch.cuda.stream(stream):
+                    device_row[first:end].copy_(src, non_blocking=False)
+            else:
+                device_row[first:end].copy_(src)
+        return first, end
 
     def close(self):
         if self.handle:

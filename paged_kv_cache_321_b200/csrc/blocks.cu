@@ -55,6 +55,9 @@ struct kvp_seq {
     std::vector<std::vector<int>> ids;      // [layer][block index]
     std::vector<std::vector<char>> owned;   // [layer][block index]: 0 = borrowed
     int computed = 0, written = 0;
+    uint64_t epoch = 0;                     // bumped whenever the blocks are replaced
+    std::vector<uint64_t> synced_epoch;     // [layer]: epoch of the last delta (~0: never)
+    std::vector<int> synced;                // [layer]: entries handed out by the last delta
 };
 
 namespace {
@@ -188,6 +191,7 @@ void free_all(kvp_seq *s)
     s->tokens.clear();
     s->hashes.clear();
     s->computed = s->written = 0;
+    ++s->epoch;
 }
 
 }  // namespace
@@ -250,6 +254,8 @@ extern "C" int kvp_seq_create(kvp_blocks *p, kvp_seq **out)
     s->pool = p;
     s->ids.resize(p->num_layers);
     s->owned.resize(p->num_layers);
+    s->synced_epoch.assign(p->num_layers, ~0ull);
+    s->synced.assign(p->num_layers, 0);
     *out = s;
     return KVP_OK;
 }
@@ -390,4 +396,26 @@ extern "C" int kvp_seq_block_table(const kvp_seq *s, int layer, int32_t *out, in
         if (owned) owned[i] = i < n ? static_cast<uint8_t>(s->owned[layer][i]) : 0;
     }
     return n;
+}
+
+extern "C" int kvp_seq_block_table_delta(kvp_seq *s, int layer, int32_t *row, int max_blocks, int *first, int *end)
+{
+    if (!s || !row || !first || !end || max_blocks < 0 || layer < 0 || layer >= static_cast<int>(s->ids.size()))
+        return set_error(KVP_EINVAL, "kvp_seq_block_table_delta: bad arguments");
+    std::lock_guard<std::mutex> lock(s->pool->mu);
+    const std::vector<int> &ids = s->ids[layer];
+    const int n = static_cast<int>(ids.size());
+    if (n > max_blocks) return set_error(KVP_ERANGE, "sequence holds %d blocks, row has %d entries", n, max_blocks);
+    if (s->synced_epoch[layer] != s->epoch) {  // first call, or the blocks were replaced: the whole row
+        for (int i = 0; i < max_blocks; ++i) row[i] = i < n ? ids[i] : -1;
+        *first = 0, *end = max_blocks;
+    } else if (n > s->synced[layer]) {  // growth: only the new entries
+        for (int i = s->synced[layer]; i < n; ++i) row[i] = ids[i];
+        *first = s->synced[layer], *end = n;
+    } else {
+        *first = *end = 0;
+    }
+    s->synced_epoch[layer] = s->epoch;
+    s->synced[layer] = n;
+    return KVP_OK;
 }

@@ -7,6 +7,7 @@ Commit publishes completed blocks)."""
 
 import random
 
+import numpy as np
 import pytest
 
 import paged_kv_cache_321_b200 as K
@@ -111,6 +112,7 @@ def test_library_matches_model_on_random_request_streams(seed):
     m = OB.PoolModel(nl, nb, bs, 64)
     seqs = [b.sequence() for _ in range(3)]
     mseqs = [OB.SeqModel(m) for _ in range(3)]
+    mirrors = {(j, l): np.full(nb, 7777, np.int32) for j in range(3) for l in range(nl)}
     prefixes = [[rng.randrange(5) for _ in range(rng.randrange(1, 20))] for _ in range(3)]
     for _ in range(300):
         i = rng.randrange(3)
@@ -148,6 +150,12 @@ def test_library_matches_model_on_random_request_streams(seed):
             s.free()
         for j in range(3):
             assert _state(seqs[j], nl) == _mstate(mseqs[j], nl), (seed, j)
+            for l in range(nl):
+                if rng.random() < 0.5:  # device rows synced at random moments
+                    got = seqs[j].block_table_delta(l, mirrors[j, l])
+                    assert got == mseqs[j].table_delta(l, nb), (seed, j, l)
+                    ids = seqs[j].block_table(l, nb)[0]
+                    assert mirrors[j, l].tolist() == ids
         for l in range(nl):
             assert b.counts(l) == m.counts(l)
             for blk in range(nb):
@@ -171,4 +179,34 @@ def test_bad_arguments_are_refused():
     with pytest.raises(K.KvpError) as e:
         s.block_table(0, max_blocks=1)
     assert e.value.code == K.KVP_ERANGE
+    s.close(), b.close()
+
+
+def test_block_table_delta_uploads_only_growth():
+    # LayerDevicePtrTables' rule: a row changes only when its blocks grow
+    # (then only the new entries) or are replaced (then all of it)
+    b = K.Blocks(2, 16, 4)
+    s = b.sequence()
+    row = np.full(10, 99, np.int32)
+    s.allocate_for_tokens(list(range(9)))          # 2 full blocks (the 9th token's block comes later)
+    assert s.block_table_delta(0, row) == (0, 10)  # first call: the whole row
+    assert row.tolist() == s.block_table(0, 10)[0] and row[2:].tolist() == [-1] * 8
+    assert s.block_table_delta(0, row) == (0, 0)   # nothing changed
+    for t in (9, 10, 11):                           # completes block 2: a third block
+        s.append_token(t)
+    assert s.block_table_delta(0, row) == (2, 3)
+    s.reserve(20)                                    # 5 blocks
+    assert s.block_table_delta(0, row) == (3, 5)
+    assert row.tolist() == s.block_table(0, 10)[0]
+    # layer 1 keeps its own state: its first call is the whole row
+    row1 = np.zeros(10, np.int32)
+    assert s.block_table_delta(1, row1) == (0, 10) and row1.tolist() == s.block_table(1, 10)[0]
+    s.free()                                         # replaced: the whole row again, all -1
+    assert s.block_table_delta(0, row) == (0, 10) and row.tolist() == [-1] * 10
+    s.allocate_for_tokens([5] * 4)
+    assert s.block_table_delta(0, row) == (0, 10) and row.tolist() == s.block_table(0, 10)[0]
+    with pytest.raises(K.KvpError) as e:
+        s.block_table_delta(0, np.zeros(0, np.int32))
+    assert e.value.code == K.KVP_ERANGE
+    assert s.block_table_delta(0, row) == (0, 0)     # a refused call leaves the state alone
     s.close(), b.close()

@@ -122,3 +122,35 @@ def test_prefix_borrowing_request_matches_oracle(orc):
         s.close()
     blocks.close()
     pool.close()
+
+
+def test_device_block_tables_follow_growth():
+    # device-resident rows kept equal to the block tables by uploading only
+    # the entries that changed (the new ones on growth, all after a new prompt)
+    dev = torch.device("cuda", 0)
+    blocks = K.Blocks(2, 32, 4, 64)
+    seqs = [blocks.sequence(), blocks.sequence()]
+    M = 16
+    dev_rows = torch.full((2, 2, M), 12345, dtype=torch.int32, device=dev)  # [layer][seq][entry]
+    host = {(l, i): np.zeros(M, np.int32) for l in range(2) for i in range(2)}
+
+    def sync_and_check():
+        for l in range(2):
+            for i, s in enumerate(seqs):
+                s.sync_block_table(l, host[l, i], dev_rows[l, i])
+        torch.cuda.synchronize()
+        for l in range(2):
+            for i, s in enumerate(seqs):
+                assert dev_rows[l, i].cpu().tolist() == s.block_table(l, M)[0]
+
+    seqs[0].allocate_for_tokens(list(range(10)))
+    seqs[1].allocate_for_tokens(list(range(100, 105)))
+    sync_and_check()
+    for t in range(30):
+        seqs[t % 2].append_token(t)
+        sync_and_check()
+    seqs[0].allocate_for_tokens([1, 2, 3, 4, 5])  # a new prompt replaces the row
+    sync_and_check()
+    for s in seqs:
+        s.close()
+    blocks.close()
