@@ -225,9 +225,9 @@ __device__ __forceinline__ int tiles_of(int ctx, int window)
     return ctx > 0 ? (ctx + TT - 1) / TT - first_tile(ctx, window) : 0;
 }
 // Block-table entry of position `pos` (a ring of mbps entries with a window).
-__device__ __forceinline__ int entry_of(const Params &p, int pos)
+__device__ __forceinline__ int entry_of(const Params &p, int window, int pos)
 {
-    return p.window > 0 ? (pos / p.bs) % p.mbps : pos / p.bs;
+    return window > 0 ? (pos / p.bs) % p.mbps : pos / p.bs;
 }
 // Valid rows of the 16-key tile starting at position tb: below the context
 // end and (with a window) at or after its first key.
@@ -461,9 +461,10 @@ __device__ __forceinline__ int atomic_add_relaxed(int *addr, int v)
     return old;
 }
 
-template <int D, int G, bool BF16>
+template <int D, int G, bool BF16, bool WIN>
 __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const Params p)
 {
+    const int win = WIN ? p.window : 0;  // a compile-time 0 in the instance without a window
     using S = Shape<D, G>;
     using M = Smem<D, G>;
     constexpr int NW = S::NW;
@@ -506,7 +507,7 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
         }
     }
     __syncthreads();
-    if (warp == 0) tile_prefix(s_ctx, s_pref, s_cpref, B, Hkv, lane, p.window);
+    if (warp == 0) tile_prefix(s_ctx, s_pref, s_cpref, B, Hkv, lane, win);
     __syncthreads();
 
     grid_launch_dependents();  // the next grid may be placed (it waits for this one)
@@ -516,8 +517,8 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
     const int W = active_warps(p, total);
     const int w = blockIdx.x * NW + warp;
     if (w >= W) return;
-    const int t_begin = cost_to_tile(static_cast<int64_t>(w) * TC / W, s_ctx, s_pref, s_cpref, B, p.window);
-    const int t_end = cost_to_tile(static_cast<int64_t>(w + 1) * TC / W, s_ctx, s_pref, s_cpref, B, p.window);
+    const int t_begin = cost_to_tile(static_cast<int64_t>(w) * TC / W, s_ctx, s_pref, s_cpref, B, win);
+    const int t_end = cost_to_tile(static_cast<int64_t>(w + 1) * TC / W, s_ctx, s_pref, s_cpref, B, win);
     if (t_begin >= t_end) return;  // no CTA-wide barrier follows
 
     // barriers: [warp][stage][K, V] "tile half landed"
@@ -535,7 +536,7 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
         }
         c.t = t;
         c.r = lo;
-        c.nt = tiles_of(s_ctx[lo], p.window);
+        c.nt = tiles_of(s_ctx[lo], win);
         const int local = t - s_pref[lo];
         c.h = local / c.nt;
         c.ti = local - c.h * c.nt;
@@ -548,8 +549,8 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
                 c.h = 0;
                 do {
                     ++c.r;
-                } while (c.r < B && tiles_of(s_ctx[c.r], p.window) == 0);
-                if (c.r < B) c.nt = tiles_of(s_ctx[c.r], p.window);
+                } while (c.r < B && tiles_of(s_ctx[c.r], win) == 0);
+                if (c.r < B) c.nt = tiles_of(s_ctx[c.r], win);
             }
         }
     };
@@ -579,12 +580,12 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
             // a segment starts here: its queries are wanted when this tile is
             if (c.ti == 0 || i == 0) d_q = c.r * p.Hq + c.h * G;
             const int ctx = s_ctx[c.r];
-            const int tb = (first_tile(ctx, p.window) + c.ti) * TT;  // position of the tile's first key
-            const int blk = p.bt[static_cast<size_t>(c.r) * p.mbps + entry_of(p, tb)];
+            const int tb = (first_tile(ctx, win) + c.ti) * TT;  // position of the tile's first key
+            const int blk = p.bt[static_cast<size_t>(c.r) * p.mbps + entry_of(p, win, tb)];
             if (blk >= 0 && blk < p.num_blocks) {
                 d_off = static_cast<int64_t>(blk) * blk_stride + static_cast<int64_t>(c.h) * p.bs * D +
                         static_cast<int64_t>(tb % p.bs) * D;
-                d_nv = static_cast<int>(tile_rows(ctx, p.window, tb));
+                d_nv = static_cast<int>(tile_rows(ctx, win, tb));
             } else {
                 report(p.status, KVP_ERANGE, c.r);
             }
@@ -595,7 +596,7 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
         Cursor c;
         locate(t_begin + i, c);
         const int ctx = s_ctx[c.r];
-        const int tb = (first_tile(ctx, p.window) + c.ti) * TT;
+        const int tb = (first_tile(ctx, win) + c.ti) * TT;
         const int32_t *btr = p.bt + static_cast<size_t>(c.r) * p.mbps;
         const uint32_t bar = kbar0 + (st * 2 + half) * 8;
         uint16_t *dst = wst + st * (S::STAGE_BYTES / 2) + half * S::TILE_WORDS;
@@ -603,7 +604,7 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
         uint32_t bytes = 0;
         int nv = 0;
         for (int t = 0; t < TT && tb + t < ctx; t += p.bs) {
-            const int b = btr[entry_of(p, tb + t)];
+            const int b = btr[entry_of(p, win, tb + t)];
             if (b >= 0 && b < p.num_blocks) {
                 bytes += p.bs * D * 2;
                 nv = t + min(p.bs, ctx - tb - t);
@@ -615,14 +616,14 @@ __global__ void __launch_bounds__(Shape<D, G>::NW * 32, 1) decode_kernel(const P
         if (bytes) {
             mbar_arrive_expect_tx(bar, bytes);
             for (int t = 0; t < nv; t += p.bs) {
-                const int b = btr[entry_of(p, tb + t)];
+                const int b = btr[entry_of(p, win, tb + t)];
                 bulk_g2s_hint(smem_addr(dst + t * D), src + b * blk_stride + static_cast<size_t>(c.h) * p.bs * D,
                               p.bs * D * 2, bar, l2pol);
             }
         } else {
             mbar_arrive(bar);
         }
-        if (half == 0) nvalid[st] = nv > 0 ? static_cast<int>(tile_rows(ctx, p.window, tb) & ((1u << nv) - 1u)) : 0;
+        if (half == 0) nvalid[st] = nv > 0 ? static_cast<int>(tile_rows(ctx, win, tb) & ((1u << nv) - 1u)) : 0;
     };
     // Issues half (0: K, 1: V) of tile i (warp-relative) into stage st.
     auto issue = [&](int i, int half, int st) {
@@ -1086,11 +1087,12 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map
         : "memory");
 }
 
-template <int D, int G, bool BF16>
+template <int D, int G, bool BF16, bool WIN>
 __global__ void __launch_bounds__(TcShape<D>::NW * 32, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                      const Params p)
 {
+    const int win = WIN ? p.window : 0;  // a compile-time 0 in the instance without a window
     static_assert(G == 4 || G == 8, "the MMA rows hold 8 heads: groups of 4 use half of them");
     using S = TcShape<D>;
     using M = TcSmem<D>;
@@ -1128,7 +1130,7 @@ __global__ void __launch_bounds__(TcShape<D>::NW * 32, 1)
         }
     }
     __syncthreads();
-    if (warp == 0) tile_prefix(s_ctx, s_pref, s_cpref, B, Hkv, lane, p.window);
+    if (warp == 0) tile_prefix(s_ctx, s_pref, s_cpref, B, Hkv, lane, win);
     __syncthreads();
     grid_launch_dependents();
 
@@ -1136,8 +1138,8 @@ __global__ void __launch_bounds__(TcShape<D>::NW * 32, 1)
     const int W = active_warps(p, total);
     const int w = blockIdx.x * NW + warp;
     if (w >= W) return;
-    const int t_begin = cost_to_tile(static_cast<int64_t>(w) * TC / W, s_ctx, s_pref, s_cpref, B, p.window);
-    const int t_end = cost_to_tile(static_cast<int64_t>(w + 1) * TC / W, s_ctx, s_pref, s_cpref, B, p.window);
+    const int t_begin = cost_to_tile(static_cast<int64_t>(w) * TC / W, s_ctx, s_pref, s_cpref, B, win);
+    const int t_end = cost_to_tile(static_cast<int64_t>(w + 1) * TC / W, s_ctx, s_pref, s_cpref, B, win);
     if (t_begin >= t_end) return;  // no CTA-wide barrier follows
 
     const uint32_t kbar0 = smem_addr(&bars[warp * NST * 2]);
@@ -1154,7 +1156,7 @@ __global__ void __launch_bounds__(TcShape<D>::NW * 32, 1)
         }
         c.t = t;
         c.r = lo;
-        c.nt = tiles_of(s_ctx[lo], p.window);
+        c.nt = tiles_of(s_ctx[lo], win);
         const int local = t - s_pref[lo];
         c.h = local / c.nt;
         c.ti = local - c.h * c.nt;
@@ -1167,8 +1169,8 @@ __global__ void __launch_bounds__(TcShape<D>::NW * 32, 1)
                 c.h = 0;
                 do {
                     ++c.r;
-                } while (c.r < B && tiles_of(s_ctx[c.r], p.window) == 0);
-                if (c.r < B) c.nt = tiles_of(s_ctx[c.r], p.window);
+                } while (c.r < B && tiles_of(s_ctx[c.r], win) == 0);
+                if (c.r < B) c.nt = tiles_of(s_ctx[c.r], win);
             }
         }
     };
@@ -1193,12 +1195,12 @@ __global__ void __launch_bounds__(TcShape<D>::NW * 32, 1)
             locate(t_begin + i, c);
             if (c.ti == 0 || i == 0) d_q = c.r * p.Hq + c.h * G;
             const int ctx = s_ctx[c.r];
-            const int tb = (first_tile(ctx, p.window) + c.ti) * TT;  // position of the tile's first key
-            const int blk = p.bt[static_cast<size_t>(c.r) * p.mbps + entry_of(p, tb)];
+            const int tb = (first_tile(ctx, win) + c.ti) * TT;  // position of the tile's first key
+            const int blk = p.bt[static_cast<size_t>(c.r) * p.mbps + entry_of(p, win, tb)];
             if (blk >= 0 && blk < p.num_blocks) {
                 d_tile = blk * Hkv + c.h;
                 d_row = tb % p.bs;
-                d_nv = min(TT, ctx - tb) | (p.window > 0 ? max(0, ctx - p.window - tb) : 0) << 8;
+                d_nv = min(TT, ctx - tb) | (win > 0 ? max(0, ctx - win - tb) : 0) << 8;
             } else {
                 report(p.status, KVP_ERANGE, c.r);
             }
@@ -1271,7 +1273,7 @@ __global__ void __launch_bounds__(TcShape<D>::NW * 32, 1)
             if (lane == 0) report(p.status, KVP_ETIMEOUT, cons.r);
             return;
         }
-        const int nv = nvalid[st] & 0xFF, f0 = nvalid[st] >> 8;  // valid rows [f0, nv)
+        const int nv = nvalid[st] & 0xFF, f0 = WIN ? nvalid[st] >> 8 : 0;  // valid rows [f0, nv)
         const uint32_t kt = ring + st * S::STAGE_BYTES, vt = kt + S::HALF_BYTES;
         // ldmatrix row of this lane: matrix lane/8 covers tokens 8*(lane/16) ..
         // and the 8-column chunk (lane/8) % 2 of each 16-column step
@@ -1632,7 +1634,9 @@ static int launch(const Params &p, bool bf16, int blocks, cudaStream_t s)
 {
     const size_t smem = Smem<D, G>::total(p.B);
     if (smem > 227 * 1024) return set_error(KVP_EUNSUPPORTED, "decode: %zu bytes of shared memory", smem);
-    auto kern = bf16 ? decode_kernel<D, G, true> : decode_kernel<D, G, false>;
+    const bool win = p.window > 0;
+    auto kern = bf16 ? (win ? decode_kernel<D, G, true, true> : decode_kernel<D, G, true, false>)
+                     : (win ? decode_kernel<D, G, false, true> : decode_kernel<D, G, false, false>);
     int rc = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)),
                         "decode smem attribute");
     if (rc) return rc;
@@ -1660,7 +1664,9 @@ static int launch_tc(const Params &p, const kvp_pool *pool, int layer, bool bf16
     if ((rc = make_pool_tmap(&mk, pool->k_base + pool->layer_words * layer, pool, TT)) ||
         (rc = make_pool_tmap(&mv, pool->v_base + pool->layer_words * layer, pool, TT)))
         return rc;
-    auto kern = bf16 ? decode_tc_kernel<D, G, true> : decode_tc_kernel<D, G, false>;
+    const bool win = p.window > 0;
+    auto kern = bf16 ? (win ? decode_tc_kernel<D, G, true, true> : decode_tc_kernel<D, G, true, false>)
+                     : (win ? decode_tc_kernel<D, G, false, true> : decode_tc_kernel<D, G, false, false>);
     if ((rc = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)),
                          "decode smem attribute")))
         return rc;
