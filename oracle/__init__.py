@@ -26,8 +26,9 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fno-builtin-sin",
           "-fno-builtin-cos", "-fno-builtin-pow", "-fopenmp", "-Wall", "-shared", "-fPIC"]
 
-F16, BF16 = 1, 2
-DTYPES = {"f16": F16, "bf16": BF16}
+F16, BF16, F32 = 1, 2, 3
+DTYPES = {"f16": F16, "bf16": BF16, "f32": F32}
+POOL_NP = {"f16": np.uint16, "bf16": np.uint16, "f32": np.uint32}  # pool element storage
 OK, EINVAL, ERANGE, EOVERFLOW, EUNSUPPORTED = 0, -1, -2, -3, -4
 
 _lock = threading.Lock()
@@ -66,7 +67,7 @@ def lib():
                                         P, P, P, P, P, f32, P, i32, i32, i32, i32, P, P, P, i32, P, P, P]),
                 "orc_paged_attention": (i32, [i32, i32, i32, i32, i32, i32, i32, P, P, P, P, i32,
                                               P, P, P, P, i32, i32, i32]),
-                "orc_gather_contiguous": (i32, [i32, i32, i32, i32, i32, P, i32, P, P]),
+                "orc_gather_contiguous": (i32, [i32, i32, i32, i32, i32, P, i32, P, P, i32]),
                 "orc_dense_attention": (i32, [i32, i32, i32, i32, P, i32, P, P, P]),
                 "orc_softmax_scale": (f64, [i32]),
             }
@@ -151,7 +152,8 @@ def kv_append(*, Hq, Hkv, D, bs, kv_dtype, q, k, v, tok_req, positions, block_ta
               rope_style=0, window=0):
     """Appends T tokens into ONE layer's pools (modified in place).
 
-    pool_k / pool_v: uint16 [num_blocks, Hkv, bs, D], C-contiguous.
+    pool_k / pool_v: [num_blocks, Hkv, bs, D], C-contiguous, uint16 for the
+    16-bit types and uint32 (float32 bit patterns) for "f32".
     rope: [max_pos, R/2, 2] float32 table (R = rope_dim or D) or None.
     window > 0: block-table rows are rings (entry (p / bs) mod row length).
     Returns (status, q_out)."""
@@ -160,7 +162,7 @@ def kv_append(*, Hq, Hkv, D, bs, kv_dtype, q, k, v, tok_req, positions, block_ta
     bt = _c(block_tables, np.int32)
     S = bt.shape[0] if S is None else S
     assert pool_k.flags.c_contiguous and pool_v.flags.c_contiguous
-    assert pool_k.dtype == np.uint16 and pool_v.dtype == np.uint16
+    assert pool_k.dtype == POOL_NP[kv_dtype] and pool_v.dtype == POOL_NP[kv_dtype]
     nb = pool_k.shape[0]
     rope = _c(rope, np.float32)
     q_out = np.zeros((T, Hq * D), dtype=np.float32)
@@ -185,6 +187,8 @@ def paged_attention(*, Hq, Hkv, D, bs, kv_dtype, q, q_seq, q_pos, block_tables, 
     out = np.empty((NQ, Hq, D), dtype=np.float32)
     maxk = int(q_pos.max(initial=-1)) + 1
     w = np.zeros((NQ, Hq, max(maxk, 1)), dtype=np.float64) if want_weights else None
+    assert pool_k.dtype == POOL_NP[kv_dtype] and pool_v.dtype == POOL_NP[kv_dtype]
+    assert pool_k.flags.c_contiguous and pool_v.flags.c_contiguous
     st = lib().orc_paged_attention(NQ, Hq, Hkv, D, bs, pool_k.shape[0], DTYPES[kv_dtype], _p(q), _p(q_seq),
                                    _p(q_pos), _p(bt), bt.shape[1], _p(pool_k), _p(pool_v), _p(out), _p(w),
                                    max(maxk, 1), window, threads)
@@ -192,9 +196,13 @@ def paged_attention(*, Hq, Hkv, D, bs, kv_dtype, q, q_seq, q_pos, block_tables, 
 
 
 def gather_contiguous(*, nk, Hkv, D, bs, bt_row, pool) -> np.ndarray:
+    """Keys (or values) 0..nk-1 of one sequence as a contiguous [nk, Hkv, D]
+    copy, in the pool's element type (uint16, or uint32 for an f32 pool)."""
     bt_row = _c(bt_row, np.int32)
-    dst = np.empty((max(nk, 0), Hkv, D), dtype=np.uint16)
-    st = lib().orc_gather_contiguous(nk, Hkv, D, bs, pool.shape[0], _p(bt_row), bt_row.size, _p(pool), _p(dst))
+    assert pool.dtype in (np.uint16, np.uint32) and pool.flags.c_contiguous
+    dst = np.empty((max(nk, 0), Hkv, D), dtype=pool.dtype)
+    dt = F32 if pool.dtype == np.uint32 else F16  # only the element size matters here
+    st = lib().orc_gather_contiguous(nk, Hkv, D, bs, pool.shape[0], _p(bt_row), bt_row.size, _p(pool), _p(dst), dt)
     if st:
         raise ValueError(f"gather failed with status {st}")
     return dst
@@ -203,8 +211,8 @@ def gather_contiguous(*, nk, Hkv, D, bs, bt_row, pool) -> np.ndarray:
 def dense_attention(*, Hq, Hkv, D, kv_dtype, q, ck, cv) -> np.ndarray:
     q = _c(q, np.float32).reshape(Hq, D)
     out = np.empty((Hq, D), dtype=np.float32)
-    st = lib().orc_dense_attention(Hq, Hkv, D, DTYPES[kv_dtype], _p(q), ck.shape[0], _p(_c(ck, np.uint16)),
-                                   _p(_c(cv, np.uint16)), _p(out))
+    st = lib().orc_dense_attention(Hq, Hkv, D, DTYPES[kv_dtype], _p(q), ck.shape[0], _p(_c(ck, POOL_NP[kv_dtype])),
+                                   _p(_c(cv, POOL_NP[kv_dtype])), _p(out))
     if st:
         raise ValueError(f"dense attention failed with status {st}")
     return out

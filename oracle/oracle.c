@@ -46,7 +46,7 @@
 #include <omp.h>
 #endif
 
-enum { ORC_F16 = 1, ORC_BF16 = 2 };
+enum { ORC_F16 = 1, ORC_BF16 = 2, ORC_F32 = 3 };
 enum {
     ORC_OK = 0,
     ORC_EINVAL = -1,
@@ -145,6 +145,21 @@ uint16_t orc_f32_to_bf16(uint32_t xb)
 }
 
 uint16_t orc_convert(uint32_t xb, int dtype) { return dtype == ORC_F16 ? orc_f32_to_f16(xb) : orc_f32_to_bf16(xb); }
+
+/* Pool elements. A 16-bit pool (fp16, bf16) holds the conversion of each
+ * float32; an fp32 pool (the float32 K/V blocks the pages' paged attention
+ * also reads, runHybridAttentionBlock's f32 path) holds the float32 itself. */
+static double pool_value(const void *pool, int64_t i, int dtype)
+{
+    if (dtype == ORC_F32) return (double)bits_to_f32(((const uint32_t *)pool)[i]);
+    return orc_value16(((const uint16_t *)pool)[i], dtype);
+}
+
+static void pool_store(void *pool, int64_t i, uint32_t xb, int dtype)
+{
+    if (dtype == ORC_F32) ((uint32_t *)pool)[i] = xb;
+    else ((uint16_t *)pool)[i] = orc_convert(xb, dtype);
+}
 
 /* Converts the bit patterns start .. start+count-1 (exhaustive checks). */
 void orc_convert_range(uint64_t start, uint64_t count, int dtype, uint16_t *out)
@@ -267,7 +282,7 @@ int orc_kv_append(int T, int S, int Hq, int Hkv, int D, int bs, int num_blocks, 
                   const float *q, const float *k, const float *v, const float *q_norm_w, const float *k_norm_w,
                   float eps, const float *rope, int rope_max_pos, int rope_dim, int rope_style, int window,
                   const int32_t *tok_req, const int32_t *positions, const int32_t *block_tables, int mbps,
-                  uint16_t *pool_k, uint16_t *pool_v, float *q_out)
+                  void *pool_k, void *pool_v, float *q_out)
 {
     int status = ORC_OK;
     if (rope_dim == 0) rope_dim = D;
@@ -309,8 +324,8 @@ int orc_kv_append(int T, int S, int Hq, int Hkv, int D, int bs, int num_blocks, 
                 uint32_t kb, vb;
                 memcpy(&kb, &t0[d], 4);
                 memcpy(&vb, &vx[d], 4);
-                pool_k[slot_index(blk, h, slot, d, Hkv, bs, D)] = orc_convert(kb, dtype);
-                pool_v[slot_index(blk, h, slot, d, Hkv, bs, D)] = orc_convert(vb, dtype);
+                pool_store(pool_k, slot_index(blk, h, slot, d, Hkv, bs, D), kb, dtype);
+                pool_store(pool_v, slot_index(blk, h, slot, d, Hkv, bs, D), vb, dtype);
             }
         }
     }
@@ -328,18 +343,18 @@ int orc_kv_append(int T, int S, int Hq, int Hkv, int D, int bs, int num_blocks, 
  * of the storage (paged or contiguous). s_j = (q . k_j) * scale;
  * w_j = exp(s_j - max) / sum; out = sum_j w_j v_j; all fp64. */
 typedef struct {
-    const uint16_t *k, *v;
+    const void *k, *v;
     const int32_t *bt; /* paged: this sequence's block table row */
     int paged, Hkv, bs, D, h, dtype;
     int mbps, window;  /* paged: entry_of's ring when window > 0 */
 } kv_src;
 
-static const uint16_t *key_row(const kv_src *s, int j, const uint16_t *base)
+/* Element index of key (or value) row j. */
+static int64_t key_row(const kv_src *s, int j)
 {
     if (s->paged)
-        return base + slot_index(s->bt[entry_of(j, s->bs, s->mbps, s->window)], s->h, j % s->bs, 0, s->Hkv, s->bs,
-                                 s->D);
-    return base + ((int64_t)j * s->Hkv + s->h) * s->D; /* contiguous [nk][Hkv][D] */
+        return slot_index(s->bt[entry_of(j, s->bs, s->mbps, s->window)], s->h, j % s->bs, 0, s->Hkv, s->bs, s->D);
+    return ((int64_t)j * s->Hkv + s->h) * s->D; /* contiguous [nk][Hkv][D] */
 }
 
 /* One query head over keys j0 .. nk-1 (sbuf holds nk doubles; w_out, if
@@ -355,10 +370,10 @@ static void attend_one(const float *qrow, int j0, int nk, const kv_src *src, dou
     for (int j = 0; j < j0; ++j) sbuf[j] = 0.0;
     double m = -INFINITY;
     for (int j = j0; j < nk; ++j) {
-        const uint16_t *kr = key_row(src, j, src->k);
+        const int64_t kr = key_row(src, j);
         double acc = 0.0;
         for (int d = 0; d < D; ++d)
-            acc += (double)qrow[d] * orc_value16(kr[d], src->dtype);
+            acc += (double)qrow[d] * pool_value(src->k, kr + d, src->dtype);
         sbuf[j] = acc * scale;
         if (sbuf[j] > m) m = sbuf[j];
     }
@@ -371,8 +386,8 @@ static void attend_one(const float *qrow, int j0, int nk, const kv_src *src, dou
     if (w_out) memcpy(w_out, sbuf, sizeof(double) * nk);
     double *acc = calloc(D, sizeof(double));
     for (int j = j0; j < nk; ++j) {
-        const uint16_t *vr = key_row(src, j, src->v);
-        for (int d = 0; d < D; ++d) acc[d] += sbuf[j] * orc_value16(vr[d], src->dtype);
+        const int64_t vr = key_row(src, j);
+        for (int d = 0; d < D; ++d) acc[d] += sbuf[j] * pool_value(src->v, vr + d, src->dtype);
     }
     for (int d = 0; d < D; ++d) out[d] = (float)acc[d];
     free(acc);
@@ -396,7 +411,7 @@ double orc_softmax_scale(int D) { return (double)(float)(1.0 / sqrt((double)D));
  */
 int orc_paged_attention(int NQ, int Hq, int Hkv, int D, int bs, int num_blocks, int dtype, const float *q,
                         const int32_t *q_seq, const int32_t *q_pos, const int32_t *block_tables, int mbps,
-                        const uint16_t *pool_k, const uint16_t *pool_v, float *out, double *weights, int max_keys,
+                        const void *pool_k, const void *pool_v, float *out, double *weights, int max_keys,
                         int window, int threads)
 {
     if (Hkv <= 0 || Hq % Hkv) return ORC_EUNSUPPORTED;
@@ -438,21 +453,22 @@ int orc_paged_attention(int NQ, int Hq, int Hkv, int D, int bs, int num_blocks, 
  * built token by token through the block table (the idea of gatherKV in
  * makarna/pkg/model/arch/hybrid_decoder.go). */
 int orc_gather_contiguous(int nk, int Hkv, int D, int bs, int num_blocks, const int32_t *bt_row, int mbps,
-                          const uint16_t *pool, uint16_t *dst)
+                          const void *pool, void *dst, int dtype)
 {
+    const size_t es = dtype == ORC_F32 ? 4 : 2; /* bytes per element */
     for (int t = 0; t < nk; ++t) {
         int j = t / bs;
         if (j >= mbps || bt_row[j] < 0 || bt_row[j] >= num_blocks) return ORC_ERANGE;
         for (int h = 0; h < Hkv; ++h)
-            memcpy(dst + ((int64_t)t * Hkv + h) * D, pool + slot_index(bt_row[j], h, t % bs, 0, Hkv, bs, D),
-                   sizeof(uint16_t) * D);
+            memcpy((char *)dst + (((int64_t)t * Hkv + h) * D) * es,
+                   (const char *)pool + slot_index(bt_row[j], h, t % bs, 0, Hkv, bs, D) * es, es * D);
     }
     return ORC_OK;
 }
 
 /* Dense attention of Hq query heads over a contiguous [nk][Hkv][D] copy. */
-int orc_dense_attention(int Hq, int Hkv, int D, int dtype, const float *q, int nk, const uint16_t *ck,
-                        const uint16_t *cv, float *out)
+int orc_dense_attention(int Hq, int Hkv, int D, int dtype, const float *q, int nk, const void *ck,
+                        const void *cv, float *out)
 {
     if (Hkv <= 0 || Hq % Hkv) return ORC_EUNSUPPORTED;
     double *sbuf = malloc(sizeof(double) * (nk > 0 ? nk : 1));

@@ -14,4 +14,6 @@ from .gen import (  # noqa: F401
     make_workload,
     spec_by_name,
     NAN16,
+    NAN_BITS,
+    POOL_NP,
 )

@@ -16,7 +16,8 @@ Every input of a hot-path step is drawn here, in a fixed order, from
    (only when the spec has q/k norm).
 
 Prior cache contents stand for keys and values that earlier steps already
-wrote. They are drawn directly as 16-bit values: the float32 draw is
+wrote. They are drawn directly as 16-bit values (an f32 pool keeps the
+float32 draws as they are): the float32 draw is
 TRUNCATED onto the 16-bit grid (bf16: the upper half of the float32 word;
 fp16: exponent re-biased and the low 13 mantissa bits dropped, magnitudes
 below the fp16 normal range set to zero). Truncation is a way of drawing
@@ -25,8 +26,8 @@ tokens, which lives only in the oracle and in the CUDA kernels.
 
 Every cache slot that holds no prior token -- including the slot each new
 token is about to be appended to, the unused tail of a sequence's last block
-and every block no sequence owns -- is filled with a 16-bit quiet-NaN
-sentinel, so any stray read turns an attention output into NaN and any stray
+and every block no sequence owns -- is filled with a quiet-NaN
+sentinel of the pool's type, so any stray read turns an attention output into NaN and any stray
 write shows up as a changed sentinel.
 
 Pool layout (per layer): ``[num_blocks][Hkv][block_size][D]`` 16-bit words,
@@ -49,6 +50,8 @@ import numpy as np
 
 SEED_BASE = 20261202
 NAN16 = {"f16": 0x7E00, "bf16": 0x7FC0}
+NAN_BITS = {**NAN16, "f32": 0x7FC00000}  # unused-slot sentinel of each pool type
+POOL_NP = {"f16": np.uint16, "bf16": np.uint16, "f32": np.uint32}
 
 
 @dataclass(frozen=True)
@@ -73,7 +76,7 @@ class Spec:
     Hkv: int
     D: int
     bs: int
-    kv_dtype: str  # "f16" or "bf16"
+    kv_dtype: str  # "f16", "bf16" or "f32" (float32 pool)
     theta: float
     segments: tuple
     eps: float = 1e-6
@@ -113,7 +116,7 @@ class Workload:
     v: np.ndarray  # float32 [T, Hkv*D]
     q_norm_w: Optional[np.ndarray]  # float32 [D] or None
     k_norm_w: Optional[np.ndarray]
-    pool_k: np.ndarray  # uint16 [num_layers, num_blocks, Hkv, bs, D]
+    pool_k: np.ndarray  # uint16 (uint32 for f32) [num_layers, num_blocks, Hkv, bs, D]
     pool_v: np.ndarray
     shared_blocks: int = 0  # blocks shared inside each group (0: none)
     extra: dict = field(default_factory=dict)
@@ -127,6 +130,10 @@ class Workload:
     def prefill_seqs(self) -> np.ndarray:
         return np.nonzero(self.q_lens > 1)[0].astype(np.int32)
 
+    @property
+    def elem_bytes(self) -> int:
+        return 4 if self.spec.kv_dtype == "f32" else 2
+
     def visible_keys(self, seqs: Optional[Sequence[int]] = None) -> np.ndarray:
         """Keys the decode query of each sequence sees: its context, or the
         last `window` of it."""
@@ -138,7 +145,7 @@ class Workload:
         """Algorithmic K+V bytes one decode pass reads: every visible key and
         value element once, for every KV head."""
         sp = self.spec
-        return int(self.visible_keys(seqs).sum()) * sp.Hkv * sp.D * 2 * 2
+        return int(self.visible_keys(seqs).sum()) * sp.Hkv * sp.D * 2 * self.elem_bytes
 
     def unique_kv_read_bytes(self, seqs: Optional[Sequence[int]] = None) -> int:
         """Like kv_read_bytes but counting each physical block slot once
@@ -155,7 +162,7 @@ class Workload:
                 bid = int(self.block_tables[r, j])
                 used = min(sp.bs, n - j * sp.bs)
                 seen[bid] = max(seen.get(bid, 0), used)
-        return sum(seen.values()) * sp.Hkv * sp.D * 2 * 2
+        return sum(seen.values()) * sp.Hkv * sp.D * 2 * self.elem_bytes
 
 
 def _normal(rng: np.random.Generator, shape, scale: float) -> np.ndarray:
@@ -166,8 +173,11 @@ def _normal(rng: np.random.Generator, shape, scale: float) -> np.ndarray:
 
 
 def _truncate_to_16(x: np.ndarray, kv_dtype: str) -> np.ndarray:
-    """Draw 16-bit values by truncating float32 draws (see module doc)."""
+    """Draw 16-bit values by truncating float32 draws (see module doc); an
+    f32 pool keeps the float32 draws as they are (their bit patterns)."""
     b = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    if kv_dtype == "f32":
+        return b.copy()
     if kv_dtype == "bf16":
         return (b >> 16).astype(np.uint16)
     a = b & np.uint32(0x7FFFFFFF)
@@ -242,9 +252,9 @@ def make_workload(spec: Spec, seed_offset: Optional[int] = None) -> Workload:
 
     # 3. prior cache contents
     L = spec.num_layers
-    nan = NAN16[spec.kv_dtype]
-    pool_k = np.full((L, num_blocks, Hkv, bs, D), nan, dtype=np.uint16)
-    pool_v = np.full((L, num_blocks, Hkv, bs, D), nan, dtype=np.uint16)
+    nan = NAN_BITS[spec.kv_dtype]
+    pool_k = np.full((L, num_blocks, Hkv, bs, D), nan, dtype=POOL_NP[spec.kv_dtype])
+    pool_v = np.full((L, num_blocks, Hkv, bs, D), nan, dtype=POOL_NP[spec.kv_dtype])
     pk, pv = pool_k[spec.layer], pool_v[spec.layer]
 
     def _place(block_ids, start, kvals, vvals):
