@@ -80,3 +80,21 @@ def test_attn_config_layout_matches_the_header():
     assert (c.rope_dim, c.rope_style, c.window) == (0, K.KVP_ROPE_HALF, 0)
     assert [f[0] for f in K.AttnConfig._fields_] == ["num_heads", "num_kv_heads", "head_dim", "rope_theta",
                                                       "rms_eps", "rope_dim", "rope_style", "window"]
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("num_layers", 0, "KVP_EINVAL"), ("num_blocks", -1, "KVP_EINVAL"), ("max_seq_len", 0, "KVP_EINVAL"),
+    ("head_dim", 96, "KVP_EUNSUPPORTED"), ("block_size", 24, "KVP_EUNSUPPORTED"),
+    ("block_size", 512, "KVP_EUNSUPPORTED"), ("kv_dtype", 3, "KVP_EINVAL"),
+])
+def test_pool_config_checked_before_any_device_call(field, value, code):
+    # PagedCacheConfig's shape rules are host checks: refused with no GPU
+    import paged_kv_cache_321_b200 as K
+
+    lib = K.lib()
+    cfg = K.CacheConfig(1, 8, 128, 16, 4096, 64, K.KVP_F16, 0)
+    setattr(cfg, field, value)
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: the check comes first
+    out = ctypes.c_void_p()
+    assert lib.kv_pool_create(ctypes.byref(cfg), fake, fake, ctypes.byref(out)) == getattr(K, code)
+    assert not out.value
