@@ -243,3 +243,48 @@ def test_swa_workload_rings(orc):
             for s in range(8):
                 nan = np.all(wl.pool_k[0, blk, :, s] == 0x7FC0)
                 assert nan == ((e, s) not in written), (r, e, s)
+
+
+@pytest.mark.parametrize("n,same", [(5, True), (6, False)])
+def test_ring_chunk_limit(orc, n, same):
+    # Why a chunk appended at once must not exceed ring tokens - window + 1:
+    # appending its tokens one at a time and attending after each is the
+    # sliding layer's meaning; appending the whole chunk first gives the same
+    # result while the chunk's later keys have not overwritten a ring slot
+    # an earlier query of it still needs (W 20, ring 6 x 4 = 24 tokens:
+    # a limit of 5 tokens), and a different one beyond
+    W, bs, ring, prior, Hq, Hkv, D = 20, 4, 6, 40, 4, 2, 64
+    rng = np.random.default_rng(60)
+    N = prior + n
+    q = rng.standard_normal((N, Hq * D)).astype(f32)
+    k = rng.standard_normal((N, Hkv * D)).astype(f32)
+    v = rng.standard_normal((N, Hkv * D)).astype(f32)
+    bt = np.arange(ring, dtype=np.int32).reshape(1, ring)
+    kw = dict(Hq=Hq, Hkv=Hkv, D=D, bs=bs, kv_dtype="f16", block_tables=bt, max_seq_len=N, window=W)
+    akw = dict(Hq=Hq, Hkv=Hkv, D=D, bs=bs, kv_dtype="f16", block_tables=bt, window=W)
+
+    def fresh():
+        return np.full((ring, Hkv, bs, D), 0x7E00, np.uint16), np.full((ring, Hkv, bs, D), 0x7E00, np.uint16)
+
+    # streamed: each query attends right after its own token is appended
+    pk, pv = fresh()
+    want = []
+    for p in range(N):
+        st, qo = orc.kv_append(q=q[p:p + 1], k=k[p:p + 1], v=v[p:p + 1], tok_req=[0], positions=[p],
+                               pool_k=pk, pool_v=pv, **kw)
+        if p >= prior:
+            st, o, _ = orc.paged_attention(q=qo.reshape(1, Hq, D), q_seq=[0], q_pos=[p], pool_k=pk, pool_v=pv, **akw)
+            want.append(o[0])
+    # chunked: the prior streamed, then the n chunk tokens appended at once
+    pk, pv = fresh()
+    for p in range(prior):
+        orc.kv_append(q=q[p:p + 1], k=k[p:p + 1], v=v[p:p + 1], tok_req=[0], positions=[p], pool_k=pk, pool_v=pv,
+                      **kw)
+    st, qo = orc.kv_append(q=q[prior:], k=k[prior:], v=v[prior:], tok_req=[0] * n,
+                           positions=list(range(prior, N)), pool_k=pk, pool_v=pv, **kw)
+    st, got, _ = orc.paged_attention(q=qo.reshape(n, Hq, D), q_seq=[0] * n, q_pos=list(range(prior, N)),
+                                     pool_k=pk, pool_v=pv, **akw)
+    assert np.array_equal(got, np.array(want)) == same
+    # the refusal rule of the prefill kernel, evaluated here, agrees
+    ctx, need = N, max(0, N - n - W + 1)
+    assert (need + ring * bs <= ctx - 1) == (not same)
